@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Benchmark of the LLA decode hot path on B200 — prints ONE JSON line (rank 0).
+
+A step is one full decode step of a looped model over a batch of sequences:
+for every loop t and layer d, one LLA decode-attention call over the cached
+latents of every sequence, then one encode call that appends each sequence's
+new token (its complete loop stack) to the latent store.  Workload default:
+Ouro-1.4B shapes (D=24, T=4, H=16, d_head=128) at ratio 21.3 (r_k=16,
+r_v=32), batch 768, context 4096: a 116 GB latent store resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) each rank runs the same per-GPU workload
+on its own sequences (weak scaling, no data-path collective); the timed
+region is bracketed by a barrier and the max over ranks is reported.
+`--impl reference` times the FP64 CPU oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import lla_synth as syn  # noqa: E402
+
+METRIC = "LLA decode attn: ctx-tokens/s/GPU and achieved HBM GB/s vs peak at ρ=21.3"
+UNIT = "ctx-tokens/s"
+DEFAULT_WORKLOAD = "ouro_rho21_b768_n4096"
+# kernels the library launches per call (our own kernels only; memsets excluded)
+LAUNCHES_PER_DECODE = {"simt": 2, "tc": 3}
+LAUNCHES_PER_ENCODE = 1
+KERNEL_SOURCES = {"simt": "decode_simt.cu", "tc": "decode_tc.cu"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.CONFIGS))
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def rho_of(cfg):
+    if cfg["variant"] == 0:
+        return 2 * cfg["T"] * cfg["d_head"] / (cfg["r_k"] + cfg["r_v"])
+    return 2 * cfg["T"] * cfg["H"] * cfg["d_head"] / (cfg["r_k"] + cfg["r_v"])
+
+
+def bytes_per_call(cfg):
+    """Algorithmic bytes of one (layer, loop) decode call: the latents it must read."""
+    per_tok = (cfg["r_k"] + cfg["r_v"]) * 2 * (cfg["H"] if cfg["variant"] == 0 else 1)
+    return cfg["batch"] * cfg["context"] * per_tok
+
+
+def config_json(cfg, name, n_gpus):
+    return {"workload": name, "batch_per_gpu": cfg["batch"], "context": cfg["context"], "D": cfg["D"], "T": cfg["T"],
+            "H": cfg["H"], "d_head": cfg["d_head"], "r_k": cfg["r_k"], "r_v": cfg["r_v"],
+            "variant": "per-head" if cfg["variant"] == 0 else "2d", "rho": round(rho_of(cfg), 3),
+            "step": f"{cfg['T']}x{cfg['D']} decode calls + 1 encode append",
+            "l2": "inputs larger than L2 (latent store >> 126 MB), no flush",
+            "parallelism": f"{n_gpus} replica(s), sequences sharded per GPU"}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample_rate(cfg, seconds, n_seq=2):
+    """ctx-tokens/s of the FP64 oracle on a bounded sample: one (layer, loop) call, n_seq sequences."""
+    from oracle import lla_oracle as O
+
+    T, H, d, rk, rv, N = cfg["T"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"], cfg["context"]
+    codec1 = syn.seeded_codec(dict(cfg, D=1), "bench/cpu")
+    if cfg["variant"] == 0:
+        cK = syn.round_bf16(syn.gaussian("bench/cpu/cK", (n_seq, N, H, rk)))
+        cV = syn.round_bf16(syn.gaussian("bench/cpu/cV", (n_seq, N, H, rv)))
+        fn = O.lla_decode
+        muK, muV = codec1["mu_k"][0].reshape(H, T, d), codec1["mu_v"][0].reshape(H, T, d)
+    else:
+        cK = syn.round_bf16(syn.gaussian("bench/cpu/cK", (n_seq, N, rk)))
+        cV = syn.round_bf16(syn.gaussian("bench/cpu/cV", (n_seq, N, rv)))
+        fn = O.lla_decode_2d
+        muK, muV = codec1["mu_k"][0].reshape(T, H, d), codec1["mu_v"][0].reshape(T, H, d)
+    q = syn.gaussian("bench/cpu/q", (n_seq, H, d))
+    lens = np.full(n_seq, N)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        fn(q, cK, cV, muK, codec1["w_up_k"][0], muV, codec1["w_up_v"][0], reps % T, lens, lens, 1 / math.sqrt(d),
+           cfg["rope_base"])
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    cores = len(os.sched_getaffinity(0))
+    return reps * n_seq * N / el, cores, (f"{reps} oracle calls x {n_seq} sequences x {N} tokens x {H} heads "
+                                         f"(one layer, loop t = call mod T), {el:.1f} s")
+
+
+def run_reference(a, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rates = []
+    sample = ""
+    for i in range(a.warmup + a.steps):
+        r, cores, sample = oracle_sample_rate(cfg, 0.0, n_seq=2)
+        if i >= a.warmup:
+            rates.append(r)
+    value = statistics.median(rates)
+    per_step_tokens = 2 * cfg["context"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": per_step_tokens / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, a.workload, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "each step: " + sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.out, _ = self.p.communicate(timeout=5)
+            except Exception:
+                self.p.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    src = os.path.join(ROOT, "decode_attention_lla_b200", "csrc", KERNEL_SOURCES[kernel])
+    rec = os.path.join(ROOT, "profiles", f"traffic_{kernel}.json")
+    if not (os.path.exists(src) and os.path.exists(rec)):
+        return None
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    with open(rec) as f:
+        j = json.load(f)
+    return j.get("dram_bytes_per_launch") if j.get("source_sha256") == h else None
+
+
+def run_ours(a, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import decode_attention_lla_b200 as lla
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=600))
+
+    T, D, H, d, rk, rv = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"]
+    B, N = cfg["batch"], cfg["context"]
+    cap = N + 1  # one free slot per sequence for the token appended by the step
+    tag = f"bench/{a.workload}/rank{rank}"
+    codec_np = syn.seeded_codec(cfg, f"bench/{a.workload}/codec")
+    desc = lla.Desc(D, T, H, d, rk, rv, cfg["variant"], cfg["rope_base"], cap + 1)
+    codec = lla.Codec(desc, codec_np["w_down_k"], codec_np["w_down_v"], codec_np["w_up_k"], codec_np["w_up_v"],
+                      codec_np["mu_k"], codec_np["mu_v"])
+    del codec_np
+    nbytes = lla.store_bytes(desc, B, cap)
+    store = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    syn.fill_gaussian_bf16_(store, tag + "/store")
+    q_all = torch.empty(T, D, B, H, d, dtype=torch.float32, device=dev)
+    q_all.normal_(generator=syn.torch_generator(tag + "/q", dev))
+    S = T * d if cfg["variant"] == 0 else T * H * d
+    x_shape = (B, D, H, 2, S) if cfg["variant"] == 0 else (B, D, 2, S)
+    x_new = torch.empty(x_shape, dtype=torch.bfloat16, device=dev)
+    x_new.normal_(generator=syn.torch_generator(tag + "/x", dev))
+    seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
+    tok_idx = torch.full((B,), N, dtype=torch.int32, device=dev)
+    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    qpos = torch.full((B,), N, dtype=torch.int32, device=dev)
+    out = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(codec.workspace_bytes(B, cap), dtype=torch.uint8, device=dev)
+    impl = {"auto": lla.IMPL_AUTO, "simt": lla.IMPL_SIMT, "tc": lla.IMPL_TC}[a.kernel]
+    scale = 1.0 / math.sqrt(d)
+    decode = lla.decode_attn if cfg["variant"] == 0 else lla.decode_attn_2d
+    kernel_name = a.kernel
+    if a.kernel == "auto":  # find which kernel "auto" runs
+        try:
+            lla.decode_attn(codec, store, B, cap, 0, 0, q_all[0, 0], qpos, lens, scale, out, ws, impl=lla.IMPL_TC)
+            kernel_name = "tc"
+        except lla.LLAError:
+            kernel_name = "simt"
+        impl = {"tc": lla.IMPL_TC, "simt": lla.IMPL_SIMT}[kernel_name]
+
+    def step(events=None, host=None):
+        k = 0
+        for t in range(T):
+            for layer in range(D):
+                q = q_all[t, layer]
+                if host is not None:
+                    q = host["q_dev"]
+                    q.copy_(host["q"][t, layer], non_blocking=True)
+                ev = events[k] if events is not None else None
+                lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl,
+                                events=ev)
+                if host is not None:
+                    host["out"][t, layer].copy_(out, non_blocking=True)
+                k += 1
+        if host is not None:
+            x_new.copy_(host["x"], non_blocking=True)
+        lla.encode(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B, cap)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # kernel events: one (begin, end) pair per decode call of the timed steps
+    ev_objs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(T * D)] for _ in range(a.steps)]
+    for row in ev_objs:
+        for e0, e1 in row:
+            e0.record()
+            e1.record()
+    torch.cuda.synchronize()
+    raw = [[(e0.cuda_event, e1.cuda_event) for e0, e1 in row] for row in ev_objs]
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        g0.record()
+        for s in range(a.steps):
+            step(events=raw[s])
+        g1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = g0.elapsed_time(g1)
+    kern_ms = [e0.elapsed_time(e1) for row in ev_objs for e0, e1 in row]
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    ctx_tokens_step = B * N * T * D
+    value = world * ctx_tokens_step * a.steps / (ms_max / 1e3)
+
+    # end to end through the C ABI with host buffers: q in, out back, new-token stacks in
+    host = {"q": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
+            "out": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
+            "x": torch.empty(x_shape, dtype=torch.bfloat16, pin_memory=True),
+            "q_dev": torch.empty(B, H, d, dtype=torch.float32, device=dev)}
+    host["q"].copy_(q_all.cpu())
+    host["x"].copy_(x_new.cpu())
+    step(host=host)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.e2e_steps):
+        step(host=host)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * ctx_tokens_step * a.e2e_steps / (float(e2e_ms.item()) / 1e3)
+    h2d = T * D * B * H * d * 4 + int(np.prod(x_shape)) * 2
+    d2h = T * D * B * H * d * 4
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        kmean = statistics.mean(kern_ms)
+        achieved = bytes_per_call(cfg) / (kmean / 1e3) / 1e9
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_json(cfg, a.workload, world),
+                "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": traffic_record(kernel_name),
+                             "kernel": f"lla decode ({kernel_name})", "peak_source": f"{peak_kind} hbm_gbs",
+                             "kernel_ms_mean": kmean, "kernel_ms_min": min(kern_ms),
+                             "algorithmic_bytes_per_launch": bytes_per_call(cfg)},
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "clocks": clk.summary(),
+                "gpu_launches": a.steps * (T * D * LAUNCHES_PER_DECODE[kernel_name] + LAUNCHES_PER_ENCODE)}
+        if world == 1 and not a.no_cpu_baseline:
+            v, cores, sample = oracle_sample_rate(cfg, a.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        print(json.dumps(line), flush=True)
+    codec.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    a = parse()
+    cfg = syn.CONFIGS[a.workload]
+    if a.impl == "reference":
+        return run_reference(a, cfg)
+    return run_ours(a, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,126 @@
+// Split-combine and V up-projection for LLA decode attention.
+//
+// Every split of a sequence's context leaves a record (m, l, acc[r_v]) per
+// head: its running maximum score, the sum of exp(s_j - m), and
+// sum_j exp(s_j - m) c^V_j in the r_v-dimensional latent space.  The records
+// are merged by log-sum-exp and the merged latent a = acc / l is lifted once:
+//   out = a W^V_up,t^T + mu^V_t,
+// which equals sum_j p_j v_hat_j because the normalised p_j sum to one
+// [LLA §3 eq. (3)].  An empty context (no records with l > 0) yields zeros.
+//
+// One CTA per (head, group of sequences): W^V_up,t of the head is staged in
+// shared memory once, transposed so that the threads of a warp (one output
+// dimension each) read consecutive words.
+#include <math.h>
+
+#include "lla_internal.cuh"
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kSeqPerCta = 16;
+
+struct CombineParams {
+    const float* partials;
+    const int32_t* slot_range;  // [B][2] (begin, end) or null: slots b*splits .. +splits
+    const float* w_up_v;
+    const float* mu_v;
+    float* out;
+    int B, H, T, d, r_v, layer, loop, splits, variant;
+};
+
+__global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
+    const int h = blockIdx.x;
+    const int b0 = blockIdx.y * kSeqPerCta;
+    const int tid = threadIdx.x;
+    const int d = p.d, rv = p.r_v;
+    extern __shared__ float smem[];
+    float* Wt = smem;           // [rv][d]
+    float* mu = Wt + rv * d;    // [d]
+    float* abar = mu + d;       // [rv]
+
+    size_t w_off, mu_off;
+    if (p.variant == 0) {
+        w_off = ((size_t(p.layer) * p.H + h) * p.T + p.loop) * size_t(d) * rv;
+        mu_off = (size_t(p.layer) * p.H + h) * size_t(p.T) * d + size_t(p.loop) * d;
+    } else {
+        w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(d) * rv;
+        mu_off = size_t(p.layer) * p.T * p.H * d + (size_t(p.loop) * p.H + h) * d;
+    }
+    for (int idx = tid; idx < d * rv; idx += kThreads) {
+        const int i = idx / rv, a = idx - i * rv;
+        Wt[a * d + i] = p.w_up_v[w_off + idx];
+    }
+    for (int i = tid; i < d; i += kThreads) mu[i] = p.mu_v[mu_off + i];
+    __syncthreads();
+
+    const size_t rec_len = lla_partial_floats(rv);
+    for (int b = b0; b < min(p.B, b0 + kSeqPerCta); ++b) {
+        int s0, s1;
+        if (p.slot_range) {
+            s0 = p.slot_range[2 * b];
+            s1 = p.slot_range[2 * b + 1];
+        } else {
+            s0 = b * p.splits;
+            s1 = s0 + p.splits;
+        }
+        float M = -INFINITY;
+        for (int s = s0; s < s1; ++s) M = fmaxf(M, p.partials[(size_t(s) * p.H + h) * rec_len]);
+        float L = 0.f;
+        if (M != -INFINITY)
+            for (int s = s0; s < s1; ++s) {
+                const float* rec = p.partials + (size_t(s) * p.H + h) * rec_len;
+                if (rec[0] != -INFINITY) L += rec[1] * expf(rec[0] - M);
+            }
+        for (int a = tid; a < rv; a += kThreads) {
+            float v = 0.f;
+            if (L > 0.f) {
+                for (int s = s0; s < s1; ++s) {
+                    const float* rec = p.partials + (size_t(s) * p.H + h) * rec_len;
+                    if (rec[0] != -INFINITY) v += rec[2 + a] * expf(rec[0] - M);
+                }
+                v /= L;
+            }
+            abar[a] = v;
+        }
+        __syncthreads();
+        float* o = p.out + (size_t(b) * p.H + h) * d;
+        for (int i = tid; i < d; i += kThreads) {
+            float v = 0.f;
+            if (L > 0.f) {
+                v = mu[i];
+                for (int a = 0; a < rv; ++a) v = fmaf(abar[a], Wt[a * d + i], v);
+            }
+            o[i] = v;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+lla_status lla_combine(const lla_decode_call& call, const float* partials, const int32_t* slot_range,
+                       int splits) {
+    const lla_codec_desc& ds = call.codec->desc;
+    CombineParams p;
+    p.partials = partials;
+    p.slot_range = slot_range;
+    p.w_up_v = call.codec->w_up_v;
+    p.mu_v = call.codec->mu_v;
+    p.out = call.out;
+    p.B = call.batch;
+    p.H = ds.H;
+    p.T = ds.T;
+    p.d = ds.d_head;
+    p.r_v = ds.r_v;
+    p.layer = call.layer;
+    p.loop = call.loop;
+    p.splits = splits;
+    p.variant = ds.variant;
+    const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + ds.r_v) * sizeof(float);
+    LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    dim3 grid(ds.H, (call.batch + kSeqPerCta - 1) / kSeqPerCta);
+    combine_kernel<<<grid, kThreads, smem, call.stream>>>(p);
+    LLA_CUDA_TRY(cudaGetLastError());
+    return LLA_OK;
+}

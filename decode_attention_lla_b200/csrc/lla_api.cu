@@ -1,0 +1,293 @@
+// C ABI of the LLA library: argument validation, codec ownership, dispatch.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "lla_internal.cuh"
+
+namespace {
+
+uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u) return uint16_t((u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u));
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return uint16_t(u >> 16);
+}
+
+double bf16_bits_to_double(uint16_t h) {
+    uint32_t u = uint32_t(h) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return double(f);
+}
+
+bool desc_valid(const lla_codec_desc* d) {
+    if (!d) return false;
+    if (d->D < 1 || d->T < 1 || d->H < 1 || d->d_head < 2 || (d->d_head & 1)) return false;
+    if (d->r_k < 1 || d->r_v < 1 || d->max_pos < 1) return false;
+    if (d->variant != 0 && d->variant != 1) return false;
+    if (!(d->rope_base > 1.0f) || !isfinite(d->rope_base)) return false;
+    const long long S = (long long)d->T * d->d_head * (d->variant == 1 ? d->H : 1);
+    if (d->r_k > S || d->r_v > S) return false;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+template <class T>
+lla_status dev_alloc(T** p, size_t count) {
+    *p = nullptr;
+    if (count == 0) return LLA_OK;
+    if (cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T)) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return LLA_ERR_OOM;
+    }
+    return LLA_OK;
+}
+
+void codec_free(lla_codec* c) {
+    if (!c) return;
+    void* ptrs[] = {c->w_up_k, c->w_up_v, c->mu_k, c->mu_v, c->bias_k, c->bias_v,
+                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+    delete c;
+}
+
+}  // namespace
+
+int lla_num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+extern "C" {
+
+const char* lla_status_string(lla_status s) {
+    switch (s) {
+        case LLA_OK: return "ok";
+        case LLA_ERR_INVALID_ARG: return "invalid argument";
+        case LLA_ERR_UNSUPPORTED_SHAPE: return "shape not supported by the selected kernel";
+        case LLA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+        case LLA_ERR_CUDA: return "CUDA runtime error";
+        case LLA_ERR_OOM: return "device out of memory";
+        case LLA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char* lla_version(void) { return "lla-b200 0.1"; }
+
+size_t lla_store_bytes(const lla_codec_desc* d, int batch, int max_tokens) {
+    if (!desc_valid(d) || batch < 0 || max_tokens < 0) return 0;
+    const size_t per = size_t(d->r_k + d->r_v) * (d->variant == 0 ? size_t(d->H) : 1);
+    return size_t(batch) * size_t(d->D) * size_t(max_tokens) * per * 2;
+}
+
+lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const float* w_down_k,
+                            const float* w_down_v, const float* w_up_k, const float* w_up_v,
+                            const float* mu_k, const float* mu_v, void* stream_) {
+    if (!out) return LLA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!desc_valid(desc) || !w_down_k || !w_down_v || !w_up_k || !w_up_v || !mu_k || !mu_v)
+        return LLA_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    lla_codec* c = new (std::nothrow) lla_codec();
+    if (!c) return LLA_ERR_OOM;
+    c->desc = *desc;
+    const int D = desc->D, T = desc->T, H = desc->H, d = desc->d_head, rk = desc->r_k, rv = desc->r_v;
+    const bool two_d = desc->variant == 1;
+    c->S = T * d * (two_d ? H : 1);
+    const int S = c->S;
+    const size_t groups = two_d ? size_t(D) : size_t(D) * H;  // number of (layer[, head]) codecs
+    if (cudaGetDevice(&c->device) != cudaSuccess) { delete c; return LLA_ERR_CUDA; }
+
+    lla_status st = LLA_OK;
+    const size_t nup_k = size_t(D) * T * H * d * rk, nup_v = size_t(D) * T * H * d * rv;
+    const size_t nmu = groups * S;
+    const int half = d / 2;
+    const size_t nrope = size_t(desc->max_pos) * half;
+    if ((st = dev_alloc(&c->w_up_k, nup_k)) || (st = dev_alloc(&c->w_up_v, nup_v)) ||
+        (st = dev_alloc(&c->mu_k, nmu)) || (st = dev_alloc(&c->mu_v, nmu)) ||
+        (st = dev_alloc(&c->bias_k, groups * rk)) || (st = dev_alloc(&c->bias_v, groups * rv)) ||
+        (st = dev_alloc(&c->w_down_k_t, groups * rk * S)) || (st = dev_alloc(&c->w_down_v_t, groups * rv * S)) ||
+        (st = dev_alloc(&c->rope_cos, nrope)) || (st = dev_alloc(&c->rope_sin, nrope))) {
+        codec_free(c);
+        return st;
+    }
+
+    // Host-side preparation in double precision.
+    std::vector<uint16_t> wdt_k(groups * rk * S), wdt_v(groups * rv * S);
+    std::vector<float> bias_k(groups * rk), bias_v(groups * rv);
+    auto prep = [&](const float* wd, const float* mu, int r, std::vector<uint16_t>& wdt, std::vector<float>& bias) {
+        for (size_t g = 0; g < groups; ++g) {
+            const float* W = wd + g * size_t(S) * r;
+            const float* m = mu + g * size_t(S);
+            for (int a = 0; a < r; ++a) {
+                double acc = 0.0;
+                uint16_t* row = wdt.data() + (g * r + a) * size_t(S);
+                for (int k = 0; k < S; ++k) {
+                    const uint16_t w16 = f32_to_bf16_rne(W[size_t(k) * r + a]);
+                    row[k] = w16;
+                    acc += double(m[k]) * bf16_bits_to_double(w16);
+                }
+                bias[g * r + a] = float(acc);  // b = mu W_down, from the bf16 W_down the kernel uses
+            }
+        }
+    };
+    prep(w_down_k, mu_k, rk, wdt_k, bias_k);
+    prep(w_down_v, mu_v, rv, wdt_v, bias_v);
+    std::vector<float> rc(nrope), rs(nrope);
+    for (int i = 0; i < half; ++i) {
+        const double theta = pow(double(desc->rope_base), -2.0 * i / d);
+        for (int pos = 0; pos < desc->max_pos; ++pos) {
+            const double ang = double(pos) * theta;
+            rc[size_t(pos) * half + i] = float(cos(ang));
+            rs[size_t(pos) * half + i] = float(sin(ang));
+        }
+    }
+    bool ok = cudaMemcpyAsync(c->w_up_k, w_up_k, nup_k * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_up_v, w_up_v, nup_v * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->mu_k, mu_k, nmu * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->mu_v, mu_v, nmu * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->bias_k, bias_k.data(), bias_k.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->bias_v, bias_v.data(), bias_v.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_down_k_t, wdt_k.data(), wdt_k.size() * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_down_v_t, wdt_v.data(), wdt_v.size() * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->rope_cos, rc.data(), rc.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->rope_sin, rs.data(), rs.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+    if (ok) ok = lla_build_phi_tiles(c, stream) == LLA_OK;
+    if (ok) ok = cudaStreamSynchronize(stream) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        codec_free(c);
+        return LLA_ERR_CUDA;
+    }
+    *out = c;
+    return LLA_OK;
+}
+
+lla_status lla_destroy_codec(lla_codec* c) {
+    if (!c) return LLA_OK;
+    cudaDeviceSynchronize();
+    codec_free(c);
+    return LLA_OK;
+}
+
+lla_status lla_codec_get_desc(const lla_codec* c, lla_codec_desc* out) {
+    if (!c || !out) return LLA_ERR_INVALID_ARG;
+    *out = c->desc;
+    return LLA_OK;
+}
+
+lla_status lla_encode(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                      const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
+                      int max_tokens, void* stream) {
+    if (!c || n < 0 || batch < 0 || max_tokens < 0) return LLA_ERR_INVALID_ARG;
+    if (layer_begin < 0 || num_layers < 1 || layer_begin + num_layers > c->desc.D) return LLA_ERR_INVALID_ARG;
+    if (n == 0) return LLA_OK;
+    if (!x || !seq_idx || !tok_idx || !store) return LLA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(store) || !aligned4(seq_idx) || !aligned4(tok_idx)) return LLA_ERR_ALIGNMENT;
+    return lla_encode_launch(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens,
+                             static_cast<cudaStream_t>(stream));
+}
+
+size_t lla_decode_workspace_bytes(const lla_codec* c, int batch, int max_tokens) {
+    if (!c || batch < 0 || max_tokens < 0) return 0;
+    size_t a = lla_simt_workspace_bytes(c, batch, max_tokens);
+    if (lla_tc_supported(c)) {
+        const size_t b = lla_tc_workspace_bytes(c, batch, max_tokens);
+        if (b > a) a = b;
+    }
+    return a;
+}
+
+static lla_status decode_common(int want_variant, const lla_codec* c, const uint16_t* store, int batch,
+                                int max_tokens, int layer, int loop, const float* q, const int32_t* q_pos,
+                                const int32_t* seq_lens, float scale, float* out, void* workspace,
+                                size_t workspace_bytes, const lla_decode_opts* opts, void* stream) {
+    if (!c || c->desc.variant != want_variant) return LLA_ERR_INVALID_ARG;
+    if (batch < 0 || max_tokens < 0 || layer < 0 || layer >= c->desc.D || loop < 0 || loop >= c->desc.T)
+        return LLA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return LLA_ERR_INVALID_ARG;
+    if (batch == 0) return LLA_OK;
+    if (!store || !q || !q_pos || !seq_lens || !out) return LLA_ERR_INVALID_ARG;
+    if (!workspace) return LLA_ERR_WORKSPACE;
+    if (!aligned16(store) || !aligned16(q) || !aligned16(out) || !aligned16(workspace) || !aligned4(q_pos) ||
+        !aligned4(seq_lens))
+        return LLA_ERR_ALIGNMENT;
+    if (workspace_bytes < lla_decode_workspace_bytes(c, batch, max_tokens)) return LLA_ERR_WORKSPACE;
+    const int impl = opts ? opts->impl : 0;
+    const int num_ctas = opts ? opts->num_ctas : 0;
+    if (impl < 0 || impl > 2 || num_ctas < 0) return LLA_ERR_INVALID_ARG;
+
+    lla_decode_call call;
+    call.codec = c;
+    call.store = store;
+    call.batch = batch;
+    call.max_tokens = max_tokens;
+    call.layer = layer;
+    call.loop = loop;
+    call.q = q;
+    call.q_pos = q_pos;
+    call.seq_lens = seq_lens;
+    call.scale = scale;
+    call.out = out;
+    call.workspace = static_cast<char*>(workspace);
+    call.workspace_bytes = workspace_bytes;
+    call.stream = static_cast<cudaStream_t>(stream);
+    if (opts) {
+        call.ev_begin = static_cast<cudaEvent_t>(opts->ev_begin);
+        call.ev_end = static_cast<cudaEvent_t>(opts->ev_end);
+    }
+    LLA_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(lla_ws_header), call.stream));
+    if (max_tokens == 0) {
+        LLA_CUDA_TRY(cudaMemsetAsync(out, 0, size_t(batch) * c->desc.H * c->desc.d_head * 4, call.stream));
+        return LLA_OK;
+    }
+    const bool tc_ok = lla_tc_supported(c);
+    if (impl == 2 && !tc_ok) return LLA_ERR_UNSUPPORTED_SHAPE;
+    if (impl == 2 || (impl == 0 && tc_ok)) return lla_decode_tc(call, num_ctas);
+    return lla_decode_simt(call, num_ctas);
+}
+
+lla_status lla_decode_attn(const lla_codec* c, const uint16_t* store, int batch, int max_tokens, int layer,
+                           int loop, const float* q, const int32_t* q_pos, const int32_t* seq_lens,
+                           float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_common(0, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out, workspace,
+                         workspace_bytes, nullptr, stream);
+}
+
+lla_status lla_decode_attn_2d(const lla_codec* c, const uint16_t* store, int batch, int max_tokens, int layer,
+                              int loop, const float* q, const int32_t* q_pos, const int32_t* seq_lens,
+                              float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_common(1, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out, workspace,
+                         workspace_bytes, nullptr, stream);
+}
+
+lla_status lla_decode_attn_ex(const lla_codec* c, const uint16_t* store, int batch, int max_tokens, int layer,
+                              int loop, const float* q, const int32_t* q_pos, const int32_t* seq_lens,
+                              float scale, float* out, void* workspace, size_t workspace_bytes,
+                              const lla_decode_opts* opts, void* stream) {
+    if (!c) return LLA_ERR_INVALID_ARG;
+    return decode_common(c->desc.variant, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out,
+                         workspace, workspace_bytes, opts, stream);
+}
+
+lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {
+    if (!workspace || !flags) return LLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LLA_CUDA_TRY(cudaMemcpyAsync(flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
+    LLA_CUDA_TRY(cudaStreamSynchronize(s));
+    return LLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Internal declarations shared by the LLA CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lla.h"
+
+struct lla_codec {
+    lla_codec_desc desc;
+    int S;          // stack length fed to W_down: T*d (per-head) or T*H*d (LLA-2D)
+    int device;
+    // float32 copies
+    float* w_up_k = nullptr;   // per-head [D][H][T][d][r_k];  2D [D][T][H][d][r_k]
+    float* w_up_v = nullptr;   // per-head [D][H][T][d][r_v];  2D [D][T][H][d][r_v]
+    float* mu_k = nullptr;     // per-head [D][H][S];          2D [D][S]
+    float* mu_v = nullptr;
+    float* bias_k = nullptr;   // b = mu W_down: per-head [D][H][r_k]; 2D [D][r_k]
+    float* bias_v = nullptr;
+    // bf16 W_down, transposed so that each latent dimension is one K-major row:
+    // per-head [D][H][r][S]; 2D [D][r][S]
+    uint16_t* w_down_k_t = nullptr;
+    uint16_t* w_down_v_t = nullptr;
+    // RoPE tables, filled in double precision on the host
+    float* rope_cos = nullptr;  // [max_pos][d/2]
+    float* rope_sin = nullptr;  // [max_pos][d/2]
+    // Position features Phi_j = [cos(j theta) | sin(j theta)] as bf16, one
+    // 128 x d_head tile per 128 positions, pre-arranged in the shared-memory
+    // image the tensor-core decode kernel feeds to tcgen05.mma.
+    uint16_t* phi_tiles = nullptr;
+    int phi_num_tiles = 0;
+};
+
+// Workspace header (first 256 bytes of every decode workspace).
+struct lla_ws_header {
+    uint32_t flags;      // LLA_FLAG_* bits
+    uint32_t pad[63];
+};
+
+enum : uint32_t {
+    LLA_FLAG_SEQ_LEN_CLAMPED = 1u,
+    LLA_FLAG_POS_CLAMPED = 2u,
+};
+
+// Common decode-call parameters after host validation.
+struct lla_decode_call {
+    const lla_codec* codec;
+    const uint16_t* store;
+    int batch, max_tokens, layer, loop;
+    const float* q;
+    const int32_t* q_pos;
+    const int32_t* seq_lens;
+    float scale;
+    float* out;
+    char* workspace;
+    size_t workspace_bytes;
+    cudaStream_t stream;
+    cudaEvent_t ev_begin = nullptr;  // recorded around the main attention kernel when set
+    cudaEvent_t ev_end = nullptr;
+};
+
+// ---- bf16 helpers ---------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// ---- partial (m, l, acc[r_v]) records written by the split kernels --------
+__host__ __device__ inline size_t lla_partial_floats(int r_v) { return size_t(r_v) + 2; }
+
+// ---- host-side entry points implemented in the .cu files ------------------
+size_t lla_simt_workspace_bytes(const lla_codec* c, int batch, int max_tokens);
+lla_status lla_decode_simt(const lla_decode_call& call, int splits_override);
+size_t lla_tc_workspace_bytes(const lla_codec* c, int batch, int max_tokens);
+bool lla_tc_supported(const lla_codec* c);
+lla_status lla_decode_tc(const lla_decode_call& call, int num_ctas_override);
+lla_status lla_combine(const lla_decode_call& call, const float* partials, const int32_t* slot_range,
+                       int splits);
+lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int layer_begin,
+                             int num_layers, const int32_t* seq_idx, const int32_t* tok_idx,
+                             uint16_t* store, int batch, int max_tokens, cudaStream_t stream);
+lla_status lla_build_phi_tiles(lla_codec* c, cudaStream_t stream);
+
+int lla_num_sms();
+
+#define LLA_CUDA_TRY(expr)                                   \
+    do {                                                     \
+        cudaError_t _e = (expr);                             \
+        if (_e != cudaSuccess) return LLA_ERR_CUDA;          \
+    } while (0)

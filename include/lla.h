@@ -1,0 +1,212 @@
+/*
+ * lla.h — C ABI of the B200 (sm_100a) Looped Latent Attention library.
+ *
+ * Looped Latent Attention (LLA) compresses the loop-indexed K/V cache of a
+ * weight-tied looped Transformer.  For each cached token, layer, head and axis
+ * (K or V) the T per-loop vectors x = [x_1; ...; x_T] are replaced by one
+ * latent c = (x - mu) W_down, and loop t's vector is rebuilt on read as
+ * x_hat_t = c W_up,t^T + mu_t.
+ *   Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+ *   Transformers" (O'Neill & Reid, arXiv 2607.15456), §3 eqs. (1)-(4),
+ *   "RoPE and reconstruction", "LLA-2D variant".
+ *
+ * Conventions shared by every entry point
+ *   - bf16 data is passed as raw bfloat16 bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Device pointers are the caller's: the library never frees them.  All
+ *     launches are asynchronous on `stream`.  Argument errors are detected
+ *     on the host before anything is launched, and reported as a status.
+ *   - Errors never cross the ABI as exceptions.  Device-side range problems
+ *     (a seq_len above max_tokens, a position outside the RoPE table) are
+ *     clamped and recorded in a status word inside the workspace, readable
+ *     with lla_workspace_flags().
+ *   - Device pointers used by the decode kernels must be 16-byte aligned;
+ *     otherwise LLA_ERR_ALIGNMENT.
+ */
+#ifndef LLA_B200_H
+#define LLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LLA_OK = 0,
+    LLA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, index out of range   */
+    LLA_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside what the kernels implement           */
+    LLA_ERR_ALIGNMENT = 3,         /* a device pointer is not 16-byte aligned             */
+    LLA_ERR_CUDA = 4,              /* a CUDA runtime call or kernel launch failed         */
+    LLA_ERR_OOM = 5,               /* device allocation for the codec failed              */
+    LLA_ERR_WORKSPACE = 6          /* workspace missing or smaller than required          */
+} lla_status;
+
+/* Human-readable text for a status code (static storage). */
+const char* lla_status_string(lla_status status);
+
+/* Library version string, e.g. "lla-b200 0.1". */
+const char* lla_version(void);
+
+/*
+ * Codec description.
+ *   D layers, T loops, H heads of width d_head; latent ranks r_k (keys) and
+ *   r_v (values) [LLA §3 eq. (2), "asymmetric ranks"].
+ *   variant 0 = per-head LLA: one (r_k + r_v) latent per token, layer, head.
+ *   variant 1 = LLA-2D: one (r_k + r_v) latent per token and layer decodes all
+ *               H heads [LLA §3, "LLA-2D variant"].
+ *   rope_base: RoPE base (rotate-half pairs (i, i + d_head/2), frequencies
+ *               base^(-2i/d_head)); RoPE is applied after reconstruction
+ *               [LLA §3, "RoPE and reconstruction"].
+ *   max_pos:   keys and queries may sit at positions [0, max_pos).
+ */
+typedef struct {
+    int D, T, H, d_head, r_k, r_v;
+    int variant;
+    float rope_base;
+    int max_pos;
+} lla_codec_desc;
+
+typedef struct lla_codec lla_codec; /* opaque; owns device copies of the codec */
+
+/*
+ * lla_create_codec — copy codec matrices (host, float32) to the device.
+ *   Per-head (variant 0), with S = T*d_head:
+ *     w_down_k [D][H][S][r_k], w_down_v [D][H][S][r_v]      (eq. (2))
+ *     w_up_k   [D][H][T][d_head][r_k], w_up_v [.. r_v]       (eq. (3), W_up,t)
+ *     mu_k, mu_v [D][H][S]                                   (mu; mu_t = loop slice)
+ *   LLA-2D (variant 1), with S2 = T*H*d_head, stacks ordered (loop, head, d):
+ *     w_down_k [D][S2][r_k], w_down_v [D][S2][r_v]
+ *     w_up_k   [D][T][H][d_head][r_k], w_up_v [.. r_v]
+ *     mu_k, mu_v [D][S2]
+ *   The device copy keeps W_down as bf16 (an encode GEMM operand), W_up and mu
+ *   as float32, b = mu W_down as float32, and RoPE tables built in double
+ *   precision.  Returns LLA_ERR_OOM if device memory runs out.  The call
+ *   synchronises `stream` before returning.  W_down and W_up are independent
+ *   inputs (equal only at SVD initialisation).
+ */
+lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc,
+                            const float* w_down_k, const float* w_down_v,
+                            const float* w_up_k, const float* w_up_v,
+                            const float* mu_k, const float* mu_v, void* stream);
+
+/* Free the codec's device memory (synchronous).  NULL is accepted. */
+lla_status lla_destroy_codec(lla_codec* codec);
+
+/* Copy out the description a codec was created with. */
+lla_status lla_codec_get_desc(const lla_codec* codec, lla_codec_desc* out);
+
+/*
+ * lla_store_bytes — exact size of a latent store.
+ *   Layout (bf16, no padding):
+ *     per-head: store[batch][D][max_tokens][H][r_k + r_v]
+ *     LLA-2D:   store[batch][D][max_tokens][r_k + r_v]
+ *   Within a token's (head's) row the K latent (r_k) precedes the V latent
+ *   (r_v).  Size = batch*D*max_tokens*(r_k+r_v)*H*2 bytes (per-head) or
+ *   without H (2D), so the compression ratio of eq. (4) holds exactly.
+ *   Returns 0 for an invalid description or negative sizes.
+ */
+size_t lla_store_bytes(const lla_codec_desc* desc, int batch, int max_tokens);
+
+/*
+ * lla_encode — write latents c = (x - mu) W_down into the store [LLA §3 eq. (2)].
+ *   x         device bf16, per-head: [n][num_layers][H][2][S] (axis 0 = K, 1 = V);
+ *             LLA-2D: [n][num_layers][2][S2].  Row i is the loop stack of
+ *             token i for layers layer_begin .. layer_begin+num_layers-1.
+ *   seq_idx, tok_idx  device int32 [n]: destination sequence and token slot
+ *             of row i (0 <= seq_idx < batch, 0 <= tok_idx < max_tokens; rows
+ *             out of range are skipped and flagged in *nothing*: they are
+ *             simply not written).
+ *   store     device bf16 latent store (layout of lla_store_bytes).
+ *   Accumulation is float32 from bf16 operands; the result is rounded to
+ *   bf16 (round-to-nearest-even).
+ */
+lla_status lla_encode(const lla_codec* codec, const uint16_t* x, int n,
+                      int layer_begin, int num_layers,
+                      const int32_t* seq_idx, const int32_t* tok_idx,
+                      uint16_t* store, int batch, int max_tokens, void* stream);
+
+/*
+ * lla_decode_workspace_bytes — device scratch the decode calls need for a
+ * given batch (split partials, query-side operands, status word).  Depends on
+ * the codec and batch, and on max_tokens only through the split count.
+ */
+size_t lla_decode_workspace_bytes(const lla_codec* codec, int batch, int max_tokens);
+
+/*
+ * lla_decode_attn — per-head LLA decode attention for one (layer, loop) call.
+ *   For every sequence b and head h, with n = seq_lens[b] cached tokens
+ *   (token j at RoPE position j) and the query at position q_pos[b]:
+ *     k_hat_j = c^K_j W^K_up,t^T + mu^K_t,   v_hat_j = c^V_j W^V_up,t^T + mu^V_t
+ *     s_j = softmax_scale * <RoPE_{q_pos}(q_bh), RoPE_j(k_hat_j)>
+ *     out_bh = sum_j softmax(s)_j v_hat_j          (zero when n == 0)
+ *   [LLA §3 eq. (3), "RoPE and reconstruction"].  The V side is summed in
+ *   latent space, (sum_j p_j c^V_j) W^V_up,t^T + mu^V_t, which is exact since
+ *   the normalised p_j sum to one.
+ *   store     device bf16 [batch][D][max_tokens][H][r_k + r_v]
+ *   q         device float32 [batch][H][d_head], before RoPE
+ *   q_pos     device int32 [batch]; seq_lens device int32 [batch] (<= max_tokens)
+ *   out       device float32 [batch][H][d_head]
+ *   workspace device, >= lla_decode_workspace_bytes(codec, batch, max_tokens),
+ *             16-byte aligned; the library owns its contents during the call.
+ *   Concurrent calls must use distinct workspaces.
+ */
+lla_status lla_decode_attn(const lla_codec* codec, const uint16_t* store, int batch,
+                           int max_tokens, int layer, int loop, const float* q,
+                           const int32_t* q_pos, const int32_t* seq_lens,
+                           float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * lla_decode_attn_2d — LLA-2D decode attention [LLA §3, "LLA-2D variant"].
+ *   Same arguments as lla_decode_attn; the codec must have variant 1 and the
+ *   store is [batch][D][max_tokens][r_k + r_v]: one latent per token decodes
+ *   all H heads through per-(loop, head) up-projections.
+ */
+lla_status lla_decode_attn_2d(const lla_codec* codec, const uint16_t* store, int batch,
+                              int max_tokens, int layer, int loop, const float* q,
+                              const int32_t* q_pos, const int32_t* seq_lens,
+                              float softmax_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * Kernel selection for tests and measurements.
+ *   impl: 0 = best available, 1 = CUDA-core reference kernel (no tensor
+ *         cores), 2 = tcgen05/TMA kernel (LLA_ERR_UNSUPPORTED_SHAPE when the
+ *         shape is outside it).
+ *   num_ctas: 0 = automatic; otherwise the number of context splits (impl 1)
+ *         or persistent CTAs (impl 2).  Results do not depend on it beyond
+ *         float32 rounding.
+ *   ev_begin, ev_end: optional cudaEvent_t handles (NULL = none), recorded on
+ *         `stream` immediately before and after the main attention kernel,
+ *         so a caller can time that kernel alone (the query prologue and the
+ *         split-combine launch fall outside the pair).
+ */
+typedef struct {
+    int impl;
+    int num_ctas;
+    void* ev_begin;
+    void* ev_end;
+} lla_decode_opts;
+
+lla_status lla_decode_attn_ex(const lla_codec* codec, const uint16_t* store, int batch,
+                              int max_tokens, int layer, int loop, const float* q,
+                              const int32_t* q_pos, const int32_t* seq_lens,
+                              float softmax_scale, float* out, void* workspace,
+                              size_t workspace_bytes, const lla_decode_opts* opts,
+                              void* stream);
+
+/*
+ * lla_workspace_flags — read the device status word of a decode workspace
+ * (synchronises `stream`).  Bit 0: a seq_len was above max_tokens (clamped);
+ * bit 1: a key or query position was outside [0, max_pos) (clamped).  The
+ * word is cleared at the start of every decode call.
+ */
+lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLA_B200_H */
