@@ -1,6 +1,8 @@
 """Build the LLA CUDA library (liblla_b200.so) in-tree for sm_100a.
 
-    python -m decode_attention_lla_b200.build [--force] [-v]
+    python decode_attention_lla_b200/build.py [--force] [-v]
+
+(Run it as a script: importing the package itself needs the built library.)
 
 Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (skipped when
 it is newer than its sources), then linked with ``nvcc -shared``.  The CUDA

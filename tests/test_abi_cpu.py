@@ -6,9 +6,9 @@ import re
 
 import pytest
 
-from decode_attention_lla_b200 import build as _build
+import __graft_entry__
 
-_build.build()
+__graft_entry__._build_module().build()
 
 import decode_attention_lla_b200 as lla  # noqa: E402
 import lla_synth as syn  # noqa: E402
