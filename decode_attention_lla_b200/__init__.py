@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblla_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m decode_attention_lla_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python decode_attention_lla_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -69,10 +69,11 @@ _decode = _sig("lla_decode_attn", _i, _decode_args + [_vp])
 _decode_2d = _sig("lla_decode_attn_2d", _i, _decode_args + [_vp])
 _decode_ex = _sig("lla_decode_attn_ex", _i, _decode_args + [ctypes.POINTER(DecodeOpts), _vp])
 _flags = _sig("lla_workspace_flags", _i, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp])
+_decode_noalloc = _sig("lla_decode_attn_noalloc", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp])
 
 EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy_codec", "lla_codec_get_desc",
             "lla_store_bytes", "lla_encode", "lla_decode_workspace_bytes", "lla_decode_attn",
-            "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags"]
+            "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc"]
 
 
 class LLAError(RuntimeError):
@@ -236,3 +237,13 @@ def workspace_flags(workspace, stream=None) -> int:
     f = ctypes.c_uint32(0)
     _check(_flags(_ptr(workspace), ctypes.byref(f), _stream(stream)), "lla_workspace_flags")
     return int(f.value)
+
+
+def decode_attn_noalloc(codec, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out, stream=None):
+    """lla_decode_attn_noalloc: decode without a caller workspace, for hosts that cannot allocate.
+
+    The library keeps the scratch in a fixed 8 MiB device array shared by all
+    calls on a device; calls that overlap on the GPU race on it.
+    """
+    _check(_decode_noalloc(codec.handle, _ptr(store), batch, max_tokens, layer, loop, _ptr(q), _ptr(q_pos),
+                           _ptr(seq_lens), float(scale), _ptr(out), _stream(stream)), "lla_decode_attn_noalloc")

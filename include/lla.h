@@ -205,6 +205,36 @@ lla_status lla_decode_attn_ex(const lla_codec* codec, const uint16_t* store, int
  */
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream);
 
+/*
+ * lla_decode_attn_noalloc — lla_decode_attn (or its LLA-2D form, chosen by
+ * the codec's variant) for callers that cannot allocate device memory.
+ *   The paper has no counterpart: this is a deployment convenience.  Some
+ *   hosts may not call cudaMalloc once they are running (the call can stall
+ *   every stream of the device), or have handed all device memory to their
+ *   own pool; they can pass inputs and outputs but not a workspace.  This
+ *   entry point runs the CUDA-core decode kernel and its split-combine with
+ *   their scratch in an 8 MiB array compiled into the library, which every
+ *   GPU that loads the library holds until the process exits.  It calls no
+ *   allocator of any kind.
+ *   Limit: shapes whose workspace (lla_decode_workspace_bytes of the
+ *   CUDA-core kernel: split records of batch x H x (r_v + 2) floats per
+ *   split) exceeds 8 MiB are rejected with LLA_ERR_WORKSPACE before anything
+ *   is launched.  The per-head workload with batch 768, H 16, r_v 32 needs
+ *   about 1.7 MiB.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents: the status word is cleared at the start of each call, the
+ *   split records are rewritten.  Calls that overlap on the GPU (different
+ *   streams, or different host threads without ordering) race on it.
+ *   Arguments and results are those of lla_decode_attn without the
+ *   workspace.
+ */
+lla_status lla_decode_attn_noalloc(const lla_codec* codec, const uint16_t* store, int batch,
+                                   int max_tokens, int layer, int loop, const float* q,
+                                   const int32_t* q_pos, const int32_t* seq_lens,
+                                   float softmax_scale, float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
