@@ -27,7 +27,44 @@ struct CombineParams {
     const float* mu_v;
     float* out;
     int B, H, T, d, r_v, layer, loop, splits, variant;
+    // tensor-core record layout (tc_P != null): see lla_tc_ranges
+    const int32_t* tc_P;
+    int tc_G, tc_parts, tc_hc;
 };
+
+// Record range [s0, s1) and record stride for (b, h).  In the tensor-core
+// layout, CTA c of G covers flattened tiles [c W / G, (c+1) W / G) with
+// W = parts * total; the CTA owning tile x is ((x + 1) G - 1) / W.
+__device__ __forceinline__ void record_range(const CombineParams& p, int b, int h, int& s0, int& s1, int& hrec,
+                                             int& hstride) {
+    if (p.tc_P) {
+        const int part = h / p.tc_hc;
+        hrec = h - part * p.tc_hc;
+        hstride = p.tc_hc;
+        const long long total = p.tc_P[p.B];
+        const int tiles = p.tc_P[b + 1] - p.tc_P[b];
+        if (tiles == 0 || total == 0) {
+            s0 = s1 = 0;
+            return;
+        }
+        const long long W = total * p.tc_parts;
+        const long long x0 = part * total + p.tc_P[b], x1 = x0 + tiles - 1;
+        const long long c0 = ((x0 + 1) * p.tc_G - 1) / W, c1 = ((x1 + 1) * p.tc_G - 1) / W;
+        const long long key = (long long)part * p.B + b;
+        s0 = int(4 * (key + c0));
+        s1 = int(4 * (key + c1 + 1));
+    } else if (p.slot_range) {
+        s0 = p.slot_range[2 * b];
+        s1 = p.slot_range[2 * b + 1];
+        hrec = h;
+        hstride = p.H;
+    } else {
+        s0 = b * p.splits;
+        s1 = s0 + p.splits;
+        hrec = h;
+        hstride = p.H;
+    }
+}
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     const int h = blockIdx.x;
@@ -56,27 +93,21 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
 
     const size_t rec_len = lla_partial_floats(rv);
     for (int b = b0; b < min(p.B, b0 + kSeqPerCta); ++b) {
-        int s0, s1;
-        if (p.slot_range) {
-            s0 = p.slot_range[2 * b];
-            s1 = p.slot_range[2 * b + 1];
-        } else {
-            s0 = b * p.splits;
-            s1 = s0 + p.splits;
-        }
+        int s0, s1, hr, hs;
+        record_range(p, b, h, s0, s1, hr, hs);
         float M = -INFINITY;
-        for (int s = s0; s < s1; ++s) M = fmaxf(M, p.partials[(size_t(s) * p.H + h) * rec_len]);
+        for (int s = s0; s < s1; ++s) M = fmaxf(M, p.partials[(size_t(s) * hs + hr) * rec_len]);
         float L = 0.f;
         if (M != -INFINITY)
             for (int s = s0; s < s1; ++s) {
-                const float* rec = p.partials + (size_t(s) * p.H + h) * rec_len;
+                const float* rec = p.partials + (size_t(s) * hs + hr) * rec_len;
                 if (rec[0] != -INFINITY) L += rec[1] * expf(rec[0] - M);
             }
         for (int a = tid; a < rv; a += kThreads) {
             float v = 0.f;
             if (L > 0.f) {
                 for (int s = s0; s < s1; ++s) {
-                    const float* rec = p.partials + (size_t(s) * p.H + h) * rec_len;
+                    const float* rec = p.partials + (size_t(s) * hs + hr) * rec_len;
                     if (rec[0] != -INFINITY) v += rec[2 + a] * expf(rec[0] - M);
                 }
                 v /= L;
@@ -99,12 +130,33 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
 
 }  // namespace
 
+static lla_status launch_combine(const lla_decode_call& call, CombineParams& p);
+
 lla_status lla_combine(const lla_decode_call& call, const float* partials, const int32_t* slot_range,
                        int splits) {
-    const lla_codec_desc& ds = call.codec->desc;
     CombineParams p;
     p.partials = partials;
     p.slot_range = slot_range;
+    p.splits = splits;
+    p.tc_P = nullptr;
+    p.tc_G = p.tc_parts = p.tc_hc = 0;
+    return launch_combine(call, p);
+}
+
+lla_status lla_combine_tc(const lla_decode_call& call, const float* records, const lla_tc_ranges& r) {
+    CombineParams p;
+    p.partials = records;
+    p.slot_range = nullptr;
+    p.splits = 0;
+    p.tc_P = r.P;
+    p.tc_G = r.G;
+    p.tc_parts = r.parts;
+    p.tc_hc = r.hc;
+    return launch_combine(call, p);
+}
+
+static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) {
+    const lla_codec_desc& ds = call.codec->desc;
     p.w_up_v = call.codec->w_up_v;
     p.mu_v = call.codec->mu_v;
     p.out = call.out;
@@ -115,7 +167,6 @@ lla_status lla_combine(const lla_decode_call& call, const float* partials, const
     p.r_v = ds.r_v;
     p.layer = call.layer;
     p.loop = call.loop;
-    p.splits = splits;
     p.variant = ds.variant;
     const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + ds.r_v) * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));

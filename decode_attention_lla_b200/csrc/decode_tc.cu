@@ -1,8 +1,822 @@
-// Tensor-core (tcgen05 / TMEM / TMA) LLA decode attention.  Placeholder until
-// the kernel lands: reports every shape as unsupported.
-#include "lla_internal.cuh"
+// Tensor-core (tcgen05 / TMEM / TMA) LLA decode attention for sm_100a.
+//
+// What is computed [LLA §3 eq. (3), "RoPE and reconstruction"]: for each
+// sequence b and head h at loop t,
+//   s_j = scale * < RoPE_{q_pos}(q), RoPE_j(c^K_j W^K_up,t^T + mu^K_t) >,
+//   out = sum_j softmax(s)_j (c^V_j W^V_up,t^T + mu^V_t).
+//
+// How.  With rotate-half RoPE, writing q' = scale * RoPE_{q_pos}(q) and
+// Phi_j = [cos(j theta_i) | sin(j theta_i)]_{i < d/2}, the score is bilinear:
+//   s_j = Phi_j . (M c^K_j + beta) = sum_a c^K_{j,a} G_{j,a} + G_{j,bias}
+// with G = Phi M_q, where the columns of M_q hold, for i < d/2,
+//   MA[i,a] = q'_i W[i,a] + q'_{i+d/2} W[i+d/2,a],  MB[i,a] = q'_{i+d/2} W[i,a] - q'_i W[i+d/2,a]
+// (and the same with mu in place of W[:,a] for the bias column).  The
+// reconstruction and the rotation thus collapse into one [128 x d] x [d x N]
+// tcgen05 GEMM per 128-token tile (Phi tile from a codec table, M_q built per
+// (sequence, head) by the prologue kernel), and the CUDA cores only do an
+// r_k-long dot product per (token, head), the online softmax, and the V side
+// in latent space: acc += p_j c^V_j.  The split-combine kernel lifts acc.
+//
+// Kernel structure (one CTA per SM, persistent over a flattened range of
+// (head part, sequence, 128-token tile) work):
+//   warp 0      TMA producer: M_q image per (sequence, head part), Phi tile
+//               per tile, latent tiles per (tile, head, token chunk) into a
+//               ring of shared-memory stages (mbarrier full/empty pairs).
+//   warp 1      TMEM allocator and MMA issuer: per tile and head group,
+//               d/16 tcgen05.mma (M=128, N=NG, K=16, fp16 in, fp32 out) into
+//               one of two TMEM buffers, committed to an mbarrier.
+//   warps 2-9   compute: thread = token row (its TMEM lane); two warps share a
+//               lane quarter and split the heads of each group.  Each warp
+//               keeps (m, l, acc) per head for its 32 rows and writes one
+//               record per (segment, quarter, head) for the combine kernel.
+// Every wait is bounded (see sm100.cuh); a timeout sets a status bit.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <math.h>
+#include <string.h>
 
-bool lla_tc_supported(const lla_codec*) { return false; }
-size_t lla_tc_workspace_bytes(const lla_codec*, int, int) { return 0; }
-lla_status lla_decode_tc(const lla_decode_call&, int) { return LLA_ERR_UNSUPPORTED_SHAPE; }
-lla_status lla_build_phi_tiles(lla_codec*, cudaStream_t) { return LLA_OK; }
+#include <mutex>
+#include <vector>
+
+#include "lla_internal.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTile = 128;
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = 32 * (2 + kComputeWarps);
+constexpr int kSmemLimit = 232448;  // 227 KB per CTA
+constexpr int kMaxCtas = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kFlagTimeout = 4u;
+
+constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <int DH_, int RK_, int RV_, int H_>
+struct Cfg {
+    static constexpr int DH = DH_, RK = RK_, RV = RV_, H = H_;
+    static constexpr int ROW = RK + RV;
+    // heads per TMEM group: as many as fit N <= 256 (even, dividing H)
+    static constexpr int HG = (16 * (RK + 1) <= 240 && H % 16 == 0) ? 16
+                              : (8 * (RK + 1) <= 240 && H % 8 == 0) ? 8
+                              : (4 * (RK + 1) <= 240 && H % 4 == 0) ? 4 : 2;
+    static constexpr int NG = round_up(HG * RK + HG, 16);
+    static constexpr int MQ_GROUP_BYTES = NG * DH * 2;
+    static constexpr int GPC_MAX = (110 * 1024) / MQ_GROUP_BYTES;  // resident M_q budget ~110 KB
+    static constexpr int GPC = (H / HG) <= GPC_MAX ? (H / HG) : ((H / HG) % 2 == 0 && GPC_MAX >= 2 ? 2 : 1);
+    static constexpr int HC = HG * GPC;  // heads per CTA work item
+    static constexpr int PARTS = H / HC;
+    static constexpr int MQ_BYTES = GPC * MQ_GROUP_BYTES;
+    static constexpr int PHI_BYTES = kTile * DH * 2;
+    static constexpr int TOKS = (ROW * 2 * 128 <= 16384) ? 128 : (ROW * 2 * 64 <= 16384) ? 64 : 32;
+    static constexpr int CHUNKS = kTile / TOKS;
+    static constexpr int STAGE_BYTES = TOKS * ROW * 2;
+    static constexpr int BAR_BYTES = 1024;
+    static constexpr int FIXED = 1024 /*align slack*/ + PHI_BYTES + MQ_BYTES + BAR_BYTES;
+    static constexpr int NST_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
+    static constexpr int NST = NST_RAW > 32 ? 32 : NST_RAW;
+    static constexpr int SMEM = FIXED + NST * STAGE_BYTES;
+    static constexpr int HPW = HC / 2;  // heads per compute warp
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int BUF_COLS = 256;
+    static constexpr uint32_t IDESC = idesc_f16_f32(128, NG);
+    // V-side lane mapping
+    static constexpr bool VQUAD = (RV == 32 || RV == 64 || RV == 128);
+    static constexpr int VAL = VQUAD ? RV / 4 : 32;          // lanes along the latent dimension
+    static constexpr int VTL = 32 / VAL;                      // token sub-lanes
+    static constexpr int VPL = VQUAD ? 4 : RV / 32;           // accumulators per lane per head
+    static_assert(DH % 64 == 0 && DH <= 256, "d_head must be a multiple of 64");
+    static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
+    static_assert(H % HC == 0 && HC % 2 == 0 && HG % 2 == 0, "head split");
+    static_assert(NG <= BUF_COLS, "TMEM buffer");
+    static_assert(NST >= 2, "stages");
+    static_assert(SMEM <= kSmemLimit, "shared memory");
+    static_assert((ROW * 2) % 16 == 0, "TMA row stride");
+};
+
+struct TcParams {
+    const uint16_t* phi_tiles;   // codec Phi table, one PHI_BYTES image per 128 positions
+    const uint8_t* mq;           // prologue output: M_q images per (part, sequence)
+    const int32_t* P;            // tile prefix per sequence [B+1]
+    const int32_t* lens;         // clamped lengths [B]
+    const float* inv_scale;      // per (b, h): log2(e) / M_q scale
+    float* records;              // [(G + PARTS*B)][4][HC][RV+2]
+    uint32_t* status;
+    int B, G;
+};
+
+// Walks the CTA's contiguous share of the flattened (part, sequence, tile) space.
+struct TileWalker {
+    const int32_t* P;
+    int B;
+    long long x, x1, total;
+    int p, b, t;
+    __device__ void init(const int32_t* P_, int B_, int G, int cta, int parts) {
+        P = P_;
+        B = B_;
+        total = P[B];
+        const long long W = total * parts;
+        x = W * cta / G;
+        x1 = W * (cta + 1) / G;
+        if (x < x1) locate();
+    }
+    __device__ void locate() {
+        p = int(x / total);
+        const long long xt = x - p * total;
+        int lo = 0, hi = B - 1;  // largest b with P[b] <= xt
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P[mid] <= xt) lo = mid;
+            else hi = mid - 1;
+        }
+        b = lo;
+        t = int(xt - P[b]);
+    }
+    __device__ bool valid() const { return x < x1; }
+    __device__ int key() const { return p * B + b; }
+    __device__ void next() {
+        ++x;
+        if (x >= x1) return;
+        ++t;
+        while (t >= P[b + 1] - P[b]) {
+            t = 0;
+            if (++b == B) {
+                b = 0;
+                ++p;
+            }
+        }
+    }
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <class C>
+__global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
+                                                                TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* phi_s = smem;
+    uint8_t* mq_s = phi_s + C::PHI_BYTES;
+    uint8_t* stage_s = mq_s + C::MQ_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stage_s + C::NST * C::STAGE_BYTES);
+    uint64_t* phi_full = bars + 0;
+    uint64_t* phi_empty = bars + 1;
+    uint64_t* mq_full = bars + 2;
+    uint64_t* mq_empty = bars + 3;
+    uint64_t* tm_full = bars + 4;   // [2]
+    uint64_t* tm_empty = bars + 6;  // [2]
+    uint64_t* st_full = bars + 8;   // [NST]
+    uint64_t* st_empty = st_full + C::NST;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(st_empty + C::NST);
+    // issued[s] = number of loads the producer has issued into stage slot s.  Consumer warps
+    // drift apart by more than the ring depth, so a parity wait alone could match the
+    // previous round of a slot; a consumer first waits until its round has been issued.
+    volatile uint32_t* issued = tmem_holder + 1;
+    if (threadIdx.x < C::NST) issued[threadIdx.x] = 0;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(phi_full, 1);
+        mbar_init(phi_empty, 1);
+        mbar_init(mq_full, 1);
+        mbar_init(mq_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(tm_full + i, 1);
+            mbar_init(tm_empty + i, kComputeWarps);
+        }
+        for (int i = 0; i < C::NST; ++i) {
+            mbar_init(st_full + i, 1);
+            mbar_init(st_empty + i, C::TOKS / 32);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    TileWalker wk;
+    wk.init(p.P, p.B, p.G, blockIdx.x, C::PARTS);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (elect_one()) {
+            prefetch_tensormap(&lat_map);
+            const uint64_t pol_stream = policy_evict_first();
+            const uint64_t pol_keep = policy_evict_last();
+            uint32_t stage_k = 0, phi_n = 0, mq_n = 0;
+            int prev_key = -1;
+            bool ok = true;
+            for (; wk.valid() && ok; wk.next()) {
+                const int key = wk.key();
+                if (key != prev_key) {
+                    if (mq_n > 0 && !(ok = mbar_wait(mq_empty, (mq_n - 1) & 1, p.status, kFlagTimeout, 1))) break;
+                    mbar_expect_tx(mq_full, C::MQ_BYTES);
+                    const uint8_t* src = p.mq + size_t(key) * C::MQ_BYTES;
+                    for (int off = 0; off < C::MQ_BYTES; off += 32768) {
+                        const int n = C::MQ_BYTES - off < 32768 ? C::MQ_BYTES - off : 32768;
+                        bulk_g2s(mq_s + off, src + off, n, mq_full, pol_keep);
+                    }
+                    ++mq_n;
+                    prev_key = key;
+                }
+                if (phi_n > 0 && !(ok = mbar_wait(phi_empty, (phi_n - 1) & 1, p.status, kFlagTimeout, 2))) break;
+                mbar_expect_tx(phi_full, C::PHI_BYTES);
+                bulk_g2s(phi_s, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES, phi_full, pol_keep);
+                ++phi_n;
+                for (int hl = 0; hl < C::HC && ok; ++hl) {
+                    const int h = wk.p * C::HC + hl;
+                    for (int ch = 0; ch < C::CHUNKS; ++ch) {
+                        const uint32_t slot = stage_k % C::NST, round = stage_k / C::NST;
+                        if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
+                            break;
+                        mbar_expect_tx(st_full + slot, C::STAGE_BYTES);
+                        tma_load_4d(stage_s + size_t(slot) * C::STAGE_BYTES, &lat_map, 0, h,
+                                    wk.t * kTile + ch * C::TOKS, wk.b, st_full + slot, pol_stream);
+                        __threadfence_block();  // the armed barrier phase precedes the published round
+                        issued[slot] = round + 1;
+                        ++stage_k;
+                    }
+                }
+            }
+            // No copy may still be in flight when the CTA exits.
+            for (uint32_t s = 0; s < C::NST && s < stage_k; ++s) {
+                const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last issue into slot s
+                mbar_wait(st_full + s, (last / C::NST) & 1, p.status, kFlagTimeout, 4);
+            }
+            if (phi_n > 0) mbar_wait(phi_full, (phi_n - 1) & 1, p.status, kFlagTimeout, 5);
+            if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t phi_n = 0, mq_n = 0, gi = 0, mq_commits = 0, phi_commits = 0;
+            int prev_key = -1;
+            bool ok = true;
+            const uint32_t phi_addr = smem_u32(phi_s), mq_addr = smem_u32(mq_s);
+            for (; wk.valid() && ok; wk.next()) {
+                const int key = wk.key();
+                if (key != prev_key) {
+                    if (prev_key != -1) {
+                        mma_commit(mq_empty);
+                        ++mq_commits;
+                    }
+                    if (!(ok = mbar_wait(mq_full, mq_n & 1, p.status, kFlagTimeout, 7))) break;
+                    ++mq_n;
+                    prev_key = key;
+                }
+                if (!(ok = mbar_wait(phi_full, phi_n & 1, p.status, kFlagTimeout, 8))) break;
+                ++phi_n;
+                tc_fence_after();
+                for (int g = 0; g < C::GPC && ok; ++g) {
+                    const uint32_t buf = gi & 1, use = gi >> 1;
+                    if (use > 0 && !(ok = mbar_wait(tm_empty + buf, (use - 1) & 1, p.status, kFlagTimeout, 9))) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + buf * C::BUF_COLS;
+#pragma unroll
+                    for (int kk = 0; kk < C::DH / 16; ++kk) {
+                        const uint32_t koff = uint32_t(kk & 3) * 32;  // 16-element K step inside the 64-wide swizzle atom
+                        const uint64_t ad = sw128_kmajor_desc(phi_addr + uint32_t(kk >> 2) * (kTile * 128) + koff);
+                        const uint64_t bd = sw128_kmajor_desc(mq_addr + g * C::MQ_GROUP_BYTES +
+                                                              uint32_t(kk >> 2) * (C::NG * 128) + koff);
+                        mma_f16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(tm_full + buf);
+                    ++gi;
+                }
+                mma_commit(phi_empty);
+                ++phi_commits;
+            }
+            if (prev_key != -1) {
+                mma_commit(mq_empty);
+                ++mq_commits;
+            }
+            // The commits' arrivals land in shared memory: see them complete before the CTA exits.
+            if (phi_commits > 0) mbar_wait(phi_empty, (phi_commits - 1) & 1, p.status, kFlagTimeout, 10);
+            if (mq_commits > 0) mbar_wait(mq_empty, (mq_commits - 1) & 1, p.status, kFlagTimeout, 11);
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int cw = warp - 2;
+        const int qd = warp & 3;        // TMEM lane quarter = token rows [32 qd, 32 qd + 32)
+        const int hf = cw >> 2;         // which half of each head group
+        const int row = 32 * qd + lane;  // tile row of this thread
+        const uint32_t lane_addr = uint32_t(32 * qd) << 16;
+        const int ch = (32 * qd) / C::TOKS;              // token chunk holding this quarter
+        const int srow0 = 32 * qd - ch * C::TOKS;        // first stage row of this warp
+        constexpr int HH = C::HG / 2;                    // heads per group handled by this warp
+
+        float m[C::HPW], l[C::HPW], isc[C::HPW], acc[C::HPW][C::VPL];
+        uint32_t gi = 0, tile_n = 0;
+        int prev_key = -1, prev_p = 0;
+        bool ok = true;
+
+        auto flush = [&](int key, int part) {
+            const long long id = (long long)blockIdx.x + key;
+#pragma unroll
+            for (int hw = 0; hw < C::HPW; ++hw) {
+                const int hl = (hw / HH) * C::HG + hf * HH + (hw % HH);
+                float* rec = p.records + ((size_t(id) * 4 + qd) * C::HC + hl) * size_t(C::RV + 2);
+                const float lsum = warp_sum(l[hw]);
+                float a[C::VPL];
+#pragma unroll
+                for (int v = 0; v < C::VPL; ++v) {
+                    a[v] = acc[hw][v];
+                    for (int o = C::VAL; o < 32; o <<= 1) a[v] += __shfl_xor_sync(0xffffffffu, a[v], o);
+                }
+                if (lane == 0) {
+                    rec[0] = (m[hw] == -INFINITY) ? -INFINITY : m[hw] * kLn2;
+                    rec[1] = lsum;
+                }
+                if (C::VQUAD) {
+                    if (lane < C::VAL)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) rec[2 + 4 * lane + v] = a[v];
+                } else {
+#pragma unroll
+                    for (int v = 0; v < C::VPL; ++v) rec[2 + lane + 32 * v] = a[v];
+                }
+            }
+            (void)part;
+        };
+
+        for (; wk.valid() && ok; wk.next(), ++tile_n) {
+            const int key = wk.key();
+            if (key != prev_key) {
+                if (prev_key != -1) flush(prev_key, prev_p);
+#pragma unroll
+                for (int hw = 0; hw < C::HPW; ++hw) {
+                    const int hl = (hw / HH) * C::HG + hf * HH + (hw % HH);
+                    m[hw] = -INFINITY;
+                    l[hw] = 0.f;
+                    isc[hw] = p.inv_scale[size_t(wk.b) * C::H + wk.p * C::HC + hl];
+#pragma unroll
+                    for (int v = 0; v < C::VPL; ++v) acc[hw][v] = 0.f;
+                }
+                prev_key = key;
+                prev_p = wk.p;
+            }
+            const int valid = min(kTile, p.lens[wk.b] - wk.t * kTile);
+            const bool row_ok = row < valid;
+            const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this warp
+
+            for (int g = 0; g < C::GPC && ok; ++g) {
+                const uint32_t buf = gi & 1, use = gi >> 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(tm_full + buf, use & 1, p.status, kFlagTimeout, 12));
+                tc_fence_after();
+                const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
+#pragma unroll
+                for (int i = 0; i < HH; ++i) {
+                    const int hg = hf * HH + i;             // head within the group
+                    const int hl = g * C::HG + hg;          // head within the CTA item
+                    const int hw = g * HH + i;              // this warp's head slot
+                    const uint32_t sk = tile_n * (C::HC * C::CHUNKS) + hl * C::CHUNKS + ch;
+                    const uint32_t slot = sk % C::NST, round = sk / C::NST;
+                    ok = __all_sync(0xffffffffu, ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14));
+                    ok = __all_sync(0xffffffffu, ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13));
+                    const uint8_t* st = stage_s + size_t(slot) * C::STAGE_BYTES;
+                    const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
+
+                    // ---- score: s = c^K . G + bias
+                    float s = 0.f;
+                    {
+                        float bias;
+                        tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
+#pragma unroll
+                        for (int a0 = 0; a0 < C::RK; a0 += 16) {
+                            float gv[16];
+                            tmem_ld<16>(tcol + hg * C::RK + a0, gv);
+                            tmem_wait_ld();
+                            const uint4 u0 = *reinterpret_cast<const uint4*>(myrow + a0 * 2);
+                            const uint4 u1 = *reinterpret_cast<const uint4*>(myrow + a0 * 2 + 16);
+                            s = fmaf(bf16_lo(u0.x), gv[0], s);
+                            s = fmaf(bf16_hi(u0.x), gv[1], s);
+                            s = fmaf(bf16_lo(u0.y), gv[2], s);
+                            s = fmaf(bf16_hi(u0.y), gv[3], s);
+                            s = fmaf(bf16_lo(u0.z), gv[4], s);
+                            s = fmaf(bf16_hi(u0.z), gv[5], s);
+                            s = fmaf(bf16_lo(u0.w), gv[6], s);
+                            s = fmaf(bf16_hi(u0.w), gv[7], s);
+                            s = fmaf(bf16_lo(u1.x), gv[8], s);
+                            s = fmaf(bf16_hi(u1.x), gv[9], s);
+                            s = fmaf(bf16_lo(u1.y), gv[10], s);
+                            s = fmaf(bf16_hi(u1.y), gv[11], s);
+                            s = fmaf(bf16_lo(u1.z), gv[12], s);
+                            s = fmaf(bf16_hi(u1.z), gv[13], s);
+                            s = fmaf(bf16_lo(u1.w), gv[14], s);
+                            s = fmaf(bf16_hi(u1.w), gv[15], s);
+                        }
+                        s += bias;
+                    }
+                    // ---- online softmax in base 2
+                    const float s2 = row_ok ? s * isc[hw] : -INFINITY;
+                    const float m_new = fmaxf(m[hw], warp_max(s2));
+                    const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m[hw] - m_new);
+                    const float pj = row_ok ? fast_exp2(s2 - m_new) : 0.f;
+                    l[hw] = fmaf(l[hw], alpha, pj);
+                    m[hw] = m_new;
+#pragma unroll
+                    for (int v = 0; v < C::VPL; ++v) acc[hw][v] *= alpha;
+                    // ---- V in latent space: acc += p_j c^V_j over this warp's rows
+                    if (C::VQUAD) {
+                        const int al = lane % C::VAL;
+                        const int ts = lane / C::VAL;
+                        // interleave token sub-lanes so that the two half-warps read disjoint banks
+                        const int tsub = C::VTL == 4 ? ((ts & 1) * 2 + (ts >> 1)) : ts;
+#pragma unroll 4
+                        for (int j0 = 0; j0 < 32; j0 += C::VTL) {
+                            const int j = j0 + tsub;
+                            const float pb = __shfl_sync(0xffffffffu, pj, j);
+                            if (j < nv) {
+                                const uint2 u = *reinterpret_cast<const uint2*>(
+                                    st + size_t(srow0 + j) * (C::ROW * 2) + (C::RK + 4 * al) * 2);
+                                acc[hw][0] = fmaf(pb, bf16_lo(u.x), acc[hw][0]);
+                                acc[hw][1] = fmaf(pb, bf16_hi(u.x), acc[hw][1]);
+                                acc[hw][2] = fmaf(pb, bf16_lo(u.y), acc[hw][2]);
+                                acc[hw][3] = fmaf(pb, bf16_hi(u.y), acc[hw][3]);
+                            }
+                        }
+                    } else {
+                        for (int j = 0; j < nv; ++j) {
+                            const float pb = __shfl_sync(0xffffffffu, pj, j);
+                            const uint16_t* vr = reinterpret_cast<const uint16_t*>(
+                                st + size_t(srow0 + j) * (C::ROW * 2) + C::RK * 2);
+#pragma unroll
+                            for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[lane + 32 * v]), acc[hw][v]);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(st_empty + slot);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tm_empty + buf);
+                ++gi;
+            }
+        }
+        if (prev_key != -1) flush(prev_key, prev_p);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Prologue: tile plan, per-(sequence, head) M_q images, record initialisation.
+// ---------------------------------------------------------------------------------------------
+
+struct ProParams {
+    const float* q;
+    const int32_t* q_pos;
+    const int32_t* seq_lens;
+    const float* w_up_k;
+    const float* mu_k;
+    const float* rope_cos;
+    const float* rope_sin;
+    int32_t* P;
+    int32_t* lens;
+    float* inv_scale;
+    uint8_t* mq;
+    float* records;
+    size_t n_record_floats;
+    uint32_t* status;
+    int B, D, T, H, DH, RK, RV, HG, NG, HC, GPC, max_tokens, max_pos, layer, loop, variant;
+    float scale;
+};
+
+__global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
+    // every block helps initialise the split records to "empty" (m = -inf, l = 0)
+    {
+        const size_t rec = size_t(p.RV) + 2;
+        const size_t nrec = p.n_record_floats / rec;
+        for (size_t r = size_t(blockIdx.x) * blockDim.x + threadIdx.x; r < nrec; r += size_t(gridDim.x) * blockDim.x) {
+            p.records[r * rec] = -INFINITY;
+            p.records[r * rec + 1] = 0.f;
+        }
+    }
+    if (blockIdx.x == 0) {
+        // exclusive prefix of per-sequence tile counts (clamped lengths)
+        __shared__ int32_t carry;
+        __shared__ int32_t warp_tot[8];
+        if (threadIdx.x == 0) carry = 0;
+        __syncthreads();
+        for (int base = 0; base < p.B; base += 256) {
+            const int b = base + threadIdx.x;
+            int n = 0;
+            if (b < p.B) {
+                n = p.seq_lens[b];
+                if (n > p.max_tokens) { n = p.max_tokens; atomicOr(p.status, LLA_FLAG_SEQ_LEN_CLAMPED); }
+                if (n > p.max_pos) { n = p.max_pos; atomicOr(p.status, LLA_FLAG_POS_CLAMPED); }
+                if (n < 0) n = 0;
+                p.lens[b] = n;
+            }
+            const int tiles = (n + kTile - 1) / kTile;
+            int v = tiles;  // inclusive warp scan
+            const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += y;
+            }
+            if (lane == 31) warp_tot[w] = v;
+            __syncthreads();
+            int before = carry;
+            for (int i = 0; i < w; ++i) before += warp_tot[i];
+            if (b < p.B) p.P[b] = before + v - tiles;
+            __syncthreads();
+            if (threadIdx.x == 255) carry = before + v;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) p.P[p.B] = carry;
+        return;
+    }
+    // (b, h) block: M_q image rows of head h
+    const int bh = blockIdx.x - 1;
+    if (bh >= p.B * p.H) return;
+    const int b = bh / p.H, h = bh % p.H;
+    const int DH = p.DH, half = DH / 2, RK = p.RK;
+    __shared__ float qr[256];
+    __shared__ float red[8];
+    int qp = p.q_pos[b];
+    if (qp < 0 || qp >= p.max_pos) {
+        qp = qp < 0 ? 0 : p.max_pos - 1;
+        if (h == 0 && threadIdx.x == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
+    }
+    const float* qv = p.q + (size_t(b) * p.H + h) * DH;
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+        const float c = p.rope_cos[size_t(qp) * half + i], s = p.rope_sin[size_t(qp) * half + i];
+        const float lo = qv[i], hi = qv[i + half];
+        qr[i] = p.scale * (lo * c - hi * s);
+        qr[i + half] = p.scale * (hi * c + lo * s);
+    }
+    __syncthreads();
+    size_t w_off, mu_off;
+    if (p.variant == 0) {
+        w_off = ((size_t(p.layer) * p.H + h) * p.T + p.loop) * size_t(DH) * RK;
+        mu_off = (size_t(p.layer) * p.H + h) * size_t(p.T) * DH + size_t(p.loop) * DH;
+    } else {
+        w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(DH) * RK;
+        mu_off = size_t(p.layer) * p.T * p.H * DH + (size_t(p.loop) * p.H + h) * DH;
+    }
+    const float* W = p.w_up_k + w_off;
+    const float* mu = p.mu_k + mu_off;
+    // element (n, k) of this head's block of M_q^T: n < RK latent column, n == RK bias
+    auto value = [&](int n, int k) -> float {
+        const int i = k < half ? k : k - half;
+        const float wl = n < RK ? W[size_t(i) * RK + n] : mu[i];
+        const float wh = n < RK ? W[size_t(i + half) * RK + n] : mu[i + half];
+        return k < half ? qr[i] * wl + qr[i + half] * wh : qr[i + half] * wl - qr[i] * wh;
+    };
+    float mx = 0.f;
+    for (int e = threadIdx.x; e < (RK + 1) * DH; e += blockDim.x) mx = fmaxf(mx, fabsf(value(e / DH, e % DH)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) mx = fmaxf(mx, red[i]);
+    // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
+    int e2 = 0;
+    float scale = 1.f;
+    if (mx > 0.f && isfinite(mx)) {
+        frexpf(mx, &e2);  // mx < 2^e2
+        scale = ldexpf(1.f, 15 - e2);
+    }
+    const int part = h / p.HC, hc = h % p.HC, g = hc / p.HG, hg = hc % p.HG;
+    uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(p.GPC) * p.NG * DH * 2 + size_t(g) * p.NG * DH * 2;
+    for (int e = threadIdx.x; e < (RK + 1) * DH; e += blockDim.x) {
+        const int n = e / DH, k = e % DH;
+        const int rowi = n < RK ? hg * RK + n : p.HG * RK + hg;
+        const __half v = __float2half_rn(value(n, k) * scale);
+        *reinterpret_cast<__half*>(img + sm100::sw128_offset(rowi, k, p.NG)) = v;
+    }
+    if (hg == 0) {  // zero the group's padding rows
+        for (int e = threadIdx.x; e < (p.NG - p.HG * (RK + 1)) * DH; e += blockDim.x) {
+            const int rowi = p.HG * (RK + 1) + e / DH, k = e % DH;
+            *reinterpret_cast<__half*>(img + sm100::sw128_offset(rowi, k, p.NG)) = __float2half_rn(0.f);
+        }
+    }
+    if (threadIdx.x == 0) p.inv_scale[size_t(b) * p.H + h] = kLog2e / scale;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+struct Layout {
+    size_t off_P, off_lens, off_isc, off_mq, off_rec, total;
+};
+
+template <class C>
+Layout tc_layout(int B, int G) {
+    Layout L;
+    auto al = [](size_t x) { return (x + 1023) & ~size_t(1023); };
+    L.off_P = al(sizeof(lla_ws_header));
+    L.off_lens = al(L.off_P + size_t(B + 1) * 4);
+    L.off_isc = al(L.off_lens + size_t(B) * 4);
+    L.off_mq = al(L.off_isc + size_t(B) * C::H * 4);
+    L.off_rec = al(L.off_mq + size_t(B) * C::PARTS * C::MQ_BYTES);
+    L.total = L.off_rec + (size_t(G) + size_t(C::PARTS) * B) * 4 * C::HC * (C::RV + 2) * sizeof(float);
+    return L;
+}
+
+template <class C>
+int tc_grid(int override_ctas) {
+    int g = override_ctas > 0 ? override_ctas : lla_num_sms();
+    return g > kMaxCtas ? kMaxCtas : g;
+}
+
+template <class C>
+lla_status run_tc(const lla_decode_call& call, int num_ctas) {
+    const lla_codec* c = call.codec;
+    const int B = call.batch;
+    const int G = tc_grid<C>(num_ctas);
+    const Layout L = tc_layout<C>(B, G);
+    if (L.total > call.workspace_bytes) return LLA_ERR_WORKSPACE;
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return LLA_ERR_CUDA;
+    if ((call.max_tokens + kTile - 1) / kTile > c->phi_num_tiles) return LLA_ERR_UNSUPPORTED_SHAPE;
+
+    char* ws = call.workspace;
+    ProParams pp;
+    pp.q = call.q;
+    pp.q_pos = call.q_pos;
+    pp.seq_lens = call.seq_lens;
+    pp.w_up_k = c->w_up_k;
+    pp.mu_k = c->mu_k;
+    pp.rope_cos = c->rope_cos;
+    pp.rope_sin = c->rope_sin;
+    pp.P = reinterpret_cast<int32_t*>(ws + L.off_P);
+    pp.lens = reinterpret_cast<int32_t*>(ws + L.off_lens);
+    pp.inv_scale = reinterpret_cast<float*>(ws + L.off_isc);
+    pp.mq = reinterpret_cast<uint8_t*>(ws + L.off_mq);
+    pp.records = reinterpret_cast<float*>(ws + L.off_rec);
+    pp.n_record_floats = (L.total - L.off_rec) / sizeof(float);
+    pp.status = reinterpret_cast<uint32_t*>(ws);
+    pp.B = B;
+    pp.D = c->desc.D;
+    pp.T = c->desc.T;
+    pp.H = C::H;
+    pp.DH = C::DH;
+    pp.RK = C::RK;
+    pp.RV = C::RV;
+    pp.HG = C::HG;
+    pp.NG = C::NG;
+    pp.HC = C::HC;
+    pp.GPC = C::GPC;
+    pp.max_tokens = call.max_tokens;
+    pp.max_pos = c->desc.max_pos;
+    pp.layer = call.layer;
+    pp.loop = call.loop;
+    pp.variant = c->desc.variant;
+    pp.scale = call.scale;
+    tc_prologue_kernel<<<1 + B * C::H, 256, 0, call.stream>>>(pp);
+    LLA_CUDA_TRY(cudaGetLastError());
+
+    // Tensor map over the layer's latents: dims (row elems, head, token, sequence).
+    const size_t row_bytes = size_t(C::H) * C::ROW * 2;
+    CUtensorMap map;
+    const void* base = call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
+    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(C::H), cuuint64_t(call.max_tokens), cuuint64_t(B)};
+    cuuint64_t strides[3] = {cuuint64_t(C::ROW * 2), cuuint64_t(row_bytes),
+                             cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
+    cuuint32_t box[4] = {cuuint32_t(C::ROW), 1u, cuuint32_t(C::TOKS), 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LLA_ERR_CUDA;
+
+    TcParams tp;
+    tp.phi_tiles = c->phi_tiles;
+    tp.mq = pp.mq;
+    tp.P = pp.P;
+    tp.lens = pp.lens;
+    tp.inv_scale = pp.inv_scale;
+    tp.records = pp.records;
+    tp.status = pp.status;
+    tp.B = B;
+    tp.G = G;
+    LLA_CUDA_TRY(cudaFuncSetAttribute(tc_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    if (call.ev_begin) LLA_CUDA_TRY(cudaEventRecord(call.ev_begin, call.stream));
+    tc_decode_kernel<C><<<G, kThreads, C::SMEM, call.stream>>>(map, tp);
+    LLA_CUDA_TRY(cudaGetLastError());
+    if (call.ev_end) LLA_CUDA_TRY(cudaEventRecord(call.ev_end, call.stream));
+    lla_tc_ranges ranges;
+    ranges.P = pp.P;
+    ranges.G = G;
+    ranges.parts = C::PARTS;
+    ranges.hc = C::HC;
+    return lla_combine_tc(call, pp.records, ranges);
+}
+
+using CfgRho21 = Cfg<128, 16, 32, 16>;
+using CfgRho4 = Cfg<128, 96, 160, 16>;
+
+enum class Which { none, rho21, rho4 };
+
+Which which(const lla_codec* c) {
+    const lla_codec_desc& d = c->desc;
+    if (d.variant != 0 || d.d_head != 128 || d.H != 16) return Which::none;
+    if (d.r_k == 16 && d.r_v == 32) return Which::rho21;
+    if (d.r_k == 96 && d.r_v == 160) return Which::rho4;
+    return Which::none;
+}
+
+}  // namespace
+
+bool lla_tc_supported(const lla_codec* c) { return which(c) != Which::none && c->phi_tiles != nullptr; }
+
+size_t lla_tc_workspace_bytes(const lla_codec* c, int batch, int) {
+    switch (which(c)) {
+        case Which::rho21: return tc_layout<CfgRho21>(batch, kMaxCtas).total;
+        case Which::rho4: return tc_layout<CfgRho4>(batch, kMaxCtas).total;
+        default: return 0;
+    }
+}
+
+lla_status lla_decode_tc(const lla_decode_call& call, int num_ctas) {
+    switch (which(call.codec)) {
+        case Which::rho21: return run_tc<CfgRho21>(call, num_ctas);
+        case Which::rho4: return run_tc<CfgRho4>(call, num_ctas);
+        default: return LLA_ERR_UNSUPPORTED_SHAPE;
+    }
+}
+
+// Phi_j = [cos(j theta_i) | sin(j theta_i)], i < d/2, as fp16 in the tcgen05
+// K-major 128-byte-swizzle image, one 128-row tile per 128 positions.
+lla_status lla_build_phi_tiles(lla_codec* c, cudaStream_t stream) {
+    const int d = c->desc.d_head;
+    if (d % 64 != 0 || d > 256) return LLA_OK;  // no tensor-core path for this width
+    const int half = d / 2;
+    const int tiles = (c->desc.max_pos + kTile - 1) / kTile;
+    std::vector<__half> img(size_t(tiles) * kTile * d);
+    std::vector<double> theta(half);
+    for (int i = 0; i < half; ++i) theta[i] = pow(double(c->desc.rope_base), -2.0 * i / d);
+    for (int t = 0; t < tiles; ++t) {
+        uint8_t* tile = reinterpret_cast<uint8_t*>(img.data() + size_t(t) * kTile * d);
+        for (int r = 0; r < kTile; ++r) {
+            const double pos = double(t) * kTile + r;
+            for (int k = 0; k < d; ++k) {
+                const int i = k < half ? k : k - half;
+                const double v = k < half ? cos(pos * theta[i]) : sin(pos * theta[i]);
+                *reinterpret_cast<__half*>(tile + sm100::sw128_offset(r, k, kTile)) = __double2half(v);
+            }
+        }
+    }
+    if (cudaMalloc(&c->phi_tiles, img.size() * sizeof(__half)) != cudaSuccess) {
+        cudaGetLastError();
+        c->phi_tiles = nullptr;
+        return LLA_ERR_OOM;
+    }
+    c->phi_num_tiles = tiles;
+    if (cudaMemcpyAsync(c->phi_tiles, img.data(), img.size() * sizeof(__half), cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+        return LLA_ERR_CUDA;
+    return cudaStreamSynchronize(stream) == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}

@@ -75,6 +75,15 @@ bool lla_tc_supported(const lla_codec* c);
 lla_status lla_decode_tc(const lla_decode_call& call, int num_ctas_override);
 lla_status lla_combine(const lla_decode_call& call, const float* partials, const int32_t* slot_range,
                        int splits);
+// Record layout of the tensor-core kernel: persistent CTA c working on
+// (part p, sequence b) writes records [(c + p*B + b)][quarter 0..3][head in part].
+struct lla_tc_ranges {
+    const int32_t* P;  // per-sequence tile prefix [B+1] (device)
+    int G;             // CTAs of the decode launch
+    int parts;         // head parts (heads per part = hc)
+    int hc;
+};
+lla_status lla_combine_tc(const lla_decode_call& call, const float* records, const lla_tc_ranges& r);
 lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int layer_begin,
                              int num_layers, const int32_t* seq_idx, const int32_t* tok_idx,
                              uint16_t* store, int batch, int max_tokens, cudaStream_t stream);
