@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling runs)")
     return ap.parse_args()
 
 
@@ -319,26 +321,28 @@ def run_ours(a, cfg):
     value = world * ctx_tokens_step * a.steps / (ms_max / 1e3)
 
     # end to end through the C ABI with host buffers: q in, out back, new-token stacks in
-    host = {"q": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
-            "out": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
-            "x": torch.empty(x_shape, dtype=torch.bfloat16, pin_memory=True),
-            "q_dev": torch.empty(B, H, d, dtype=torch.float32, device=dev)}
-    host["q"].copy_(q_all.cpu())
-    host["x"].copy_(x_new.cpu())
-    step(host=host)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.e2e_steps):
+    e2e_value = None
+    if a.e2e_steps > 0:
+        host = {"q": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
+                "out": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
+                "x": torch.empty(x_shape, dtype=torch.bfloat16, pin_memory=True),
+                "q_dev": torch.empty(B, H, d, dtype=torch.float32, device=dev)}
+        host["q"].copy_(q_all.cpu())
+        host["x"].copy_(x_new.cpu())
         step(host=host)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * ctx_tokens_step * a.e2e_steps / (float(e2e_ms.item()) / 1e3)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(a.e2e_steps):
+            step(host=host)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e_value = world * ctx_tokens_step * a.e2e_steps / (float(e2e_ms.item()) / 1e3)
     h2d = T * D * B * H * d * 4 + int(np.prod(x_shape)) * 2
     d2h = T * D * B * H * d * 4
 
@@ -371,7 +375,10 @@ def run_ours(a, cfg):
 
 def main():
     a = parse()
-    cfg = syn.CONFIGS[a.workload]
+    cfg = dict(syn.CONFIGS[a.workload])
+    if a.batch or a.layers:
+        cfg.update(batch=a.batch or cfg["batch"], D=a.layers or cfg["D"])
+        a.workload = f"{a.workload}[batch={cfg['batch']},layers={cfg['D']}]"
     if a.impl == "reference":
         return run_reference(a, cfg)
     return run_ours(a, cfg)

@@ -46,13 +46,12 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;
-constexpr int kComputeWarps = 8;
-constexpr int kThreads = 32 * (2 + kComputeWarps);
 constexpr int kSmemLimit = 232448;  // 227 KB per CTA
 constexpr int kMaxCtas = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kFlagTimeout = 4u;
+constexpr int kProSeqs = 16;  // sequences per prologue block
 
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
@@ -80,7 +79,11 @@ struct Cfg {
     static constexpr int NST_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int NST = NST_RAW > 32 ? 32 : NST_RAW;
     static constexpr int SMEM = FIXED + NST * STAGE_BYTES;
-    static constexpr int HPW = HC / 2;  // heads per compute warp
+    // compute warps: WPQ per TMEM lane quarter, each taking HG / WPQ heads of every group
+    static constexpr int WPQ = HG >= 4 ? 4 : HG;
+    static constexpr int NCW = 4 * WPQ;
+    static constexpr int THREADS = 32 * (2 + NCW);
+    static constexpr int HPW = HC / WPQ;  // heads per compute warp
     static constexpr int TMEM_COLS = 512;
     static constexpr int BUF_COLS = 256;
     static constexpr uint32_t IDESC = idesc_f16_f32(128, NG);
@@ -91,7 +94,7 @@ struct Cfg {
     static constexpr int VPL = VQUAD ? 4 : RV / 32;           // accumulators per lane per head
     static_assert(DH % 64 == 0 && DH <= 256, "d_head must be a multiple of 64");
     static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
-    static_assert(H % HC == 0 && HC % 2 == 0 && HG % 2 == 0, "head split");
+    static_assert(H % HC == 0 && HG % WPQ == 0 && HG % 2 == 0, "head split");
     static_assert(NG <= BUF_COLS, "TMEM buffer");
     static_assert(NST >= 2, "stages");
     static_assert(SMEM <= kSmemLimit, "shared memory");
@@ -169,7 +172,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
+__global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
                                                                 TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
         mbar_init(mq_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(tm_full + i, 1);
-            mbar_init(tm_empty + i, kComputeWarps);
+            mbar_init(tm_empty + i, C::NCW);
         }
         for (int i = 0; i < C::NST; ++i) {
             mbar_init(st_full + i, 1);
@@ -321,14 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
         // ------------------------------------------------------------ compute warps
         const int cw = warp - 2;
         const int qd = warp & 3;        // TMEM lane quarter = token rows [32 qd, 32 qd + 32)
-        const int hf = cw >> 2;         // which half of each head group
+        const int hf = cw >> 2;         // which of the WPQ warps of this quarter
         const int row = 32 * qd + lane;  // tile row of this thread
         const uint32_t lane_addr = uint32_t(32 * qd) << 16;
         const int ch = (32 * qd) / C::TOKS;              // token chunk holding this quarter
         const int srow0 = 32 * qd - ch * C::TOKS;        // first stage row of this warp
-        constexpr int HH = C::HG / 2;                    // heads per group handled by this warp
+        constexpr int HH = C::HG / C::WPQ;               // heads per group handled by this warp
 
-        float m[C::HPW], l[C::HPW], isc[C::HPW], acc[C::HPW][C::VPL];
+        float m[C::HPW], l[C::HPW], acc[C::HPW][C::VPL];
+        const float* isc_row = p.inv_scale;  // per-(b, h) score scale, re-read from L1 when needed
         uint32_t gi = 0, tile_n = 0;
         int prev_key = -1, prev_p = 0;
         bool ok = true;
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
             const long long id = (long long)blockIdx.x + key;
 #pragma unroll
             for (int hw = 0; hw < C::HPW; ++hw) {
-                const int hl = (hw / HH) * C::HG + hf * HH + (hw % HH);
+                const int hl = (hw / HH) * C::HG + C::WPQ * (hw % HH) + hf;
                 float* rec = p.records + ((size_t(id) * 4 + qd) * C::HC + hl) * size_t(C::RV + 2);
                 const float lsum = warp_sum(l[hw]);
                 float a[C::VPL];
@@ -368,15 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
                 if (prev_key != -1) flush(prev_key, prev_p);
 #pragma unroll
                 for (int hw = 0; hw < C::HPW; ++hw) {
-                    const int hl = (hw / HH) * C::HG + hf * HH + (hw % HH);
+                    const int hl = (hw / HH) * C::HG + C::WPQ * (hw % HH) + hf;
                     m[hw] = -INFINITY;
                     l[hw] = 0.f;
-                    isc[hw] = p.inv_scale[size_t(wk.b) * C::H + wk.p * C::HC + hl];
+                    (void)hl;
 #pragma unroll
                     for (int v = 0; v < C::VPL; ++v) acc[hw][v] = 0.f;
                 }
                 prev_key = key;
                 prev_p = wk.p;
+                isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
             }
             const int valid = min(kTile, p.lens[wk.b] - wk.t * kTile);
             const bool row_ok = row < valid;
@@ -387,51 +392,49 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
                 ok = __all_sync(0xffffffffu, mbar_wait(tm_full + buf, use & 1, p.status, kFlagTimeout, 12));
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
+                // Heads of the group alternate between the two warp halves (hg = 2 i + hf), one
+                // at a time, and each latent stage is released right after use: the stages in
+                // use are adjacent in ring order and the rest of the ring keeps prefetching.
 #pragma unroll
                 for (int i = 0; i < HH; ++i) {
-                    const int hg = hf * HH + i;             // head within the group
+                    const int hg = C::WPQ * i + hf;         // head within the group
                     const int hl = g * C::HG + hg;          // head within the CTA item
                     const int hw = g * HH + i;              // this warp's head slot
                     const uint32_t sk = tile_n * (C::HC * C::CHUNKS) + hl * C::CHUNKS + ch;
                     const uint32_t slot = sk % C::NST, round = sk / C::NST;
-                    ok = __all_sync(0xffffffffu, ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14));
-                    ok = __all_sync(0xffffffffu, ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13));
+                    // score pieces from TMEM first: their latency overlaps the stage wait
+                    float gv[C::RK];
+                    float bias;
+                    tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
+#pragma unroll
+                    for (int a0 = 0; a0 < C::RK; a0 += 16) tmem_ld<16>(tcol + hg * C::RK + a0, &gv[a0]);
+                    bool w_ok = true;
+                    if (lane == 0) {
+                        w_ok = ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14);
+                        w_ok = w_ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13);
+                    }
+                    ok = __shfl_sync(0xffffffffu, w_ok, 0) && ok;
+                    __syncwarp();  // lane 0's barrier acquire covers the whole warp's reads
+                    tmem_wait_ld();
                     const uint8_t* st = stage_s + size_t(slot) * C::STAGE_BYTES;
                     const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
 
                     // ---- score: s = c^K . G + bias
-                    float s = 0.f;
-                    {
-                        float bias;
-                        tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
+                    float sa = 0.f, sb = 0.f;
 #pragma unroll
-                        for (int a0 = 0; a0 < C::RK; a0 += 16) {
-                            float gv[16];
-                            tmem_ld<16>(tcol + hg * C::RK + a0, gv);
-                            tmem_wait_ld();
-                            const uint4 u0 = *reinterpret_cast<const uint4*>(myrow + a0 * 2);
-                            const uint4 u1 = *reinterpret_cast<const uint4*>(myrow + a0 * 2 + 16);
-                            s = fmaf(bf16_lo(u0.x), gv[0], s);
-                            s = fmaf(bf16_hi(u0.x), gv[1], s);
-                            s = fmaf(bf16_lo(u0.y), gv[2], s);
-                            s = fmaf(bf16_hi(u0.y), gv[3], s);
-                            s = fmaf(bf16_lo(u0.z), gv[4], s);
-                            s = fmaf(bf16_hi(u0.z), gv[5], s);
-                            s = fmaf(bf16_lo(u0.w), gv[6], s);
-                            s = fmaf(bf16_hi(u0.w), gv[7], s);
-                            s = fmaf(bf16_lo(u1.x), gv[8], s);
-                            s = fmaf(bf16_hi(u1.x), gv[9], s);
-                            s = fmaf(bf16_lo(u1.y), gv[10], s);
-                            s = fmaf(bf16_hi(u1.y), gv[11], s);
-                            s = fmaf(bf16_lo(u1.z), gv[12], s);
-                            s = fmaf(bf16_hi(u1.z), gv[13], s);
-                            s = fmaf(bf16_lo(u1.w), gv[14], s);
-                            s = fmaf(bf16_hi(u1.w), gv[15], s);
-                        }
-                        s += bias;
+                    for (int a0 = 0; a0 < C::RK; a0 += 8) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(myrow + a0 * 2);
+                        sa = fmaf(bf16_lo(u.x), gv[a0 + 0], sa);
+                        sb = fmaf(bf16_hi(u.x), gv[a0 + 1], sb);
+                        sa = fmaf(bf16_lo(u.y), gv[a0 + 2], sa);
+                        sb = fmaf(bf16_hi(u.y), gv[a0 + 3], sb);
+                        sa = fmaf(bf16_lo(u.z), gv[a0 + 4], sa);
+                        sb = fmaf(bf16_hi(u.z), gv[a0 + 5], sb);
+                        sa = fmaf(bf16_lo(u.w), gv[a0 + 6], sa);
+                        sb = fmaf(bf16_hi(u.w), gv[a0 + 7], sb);
                     }
+                    const float s2 = row_ok ? (sa + sb + bias) * __ldg(isc_row + hl) : -INFINITY;
                     // ---- online softmax in base 2
-                    const float s2 = row_ok ? s * isc[hw] : -INFINITY;
                     const float m_new = fmaxf(m[hw], warp_max(s2));
                     const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m[hw] - m_new);
                     const float pj = row_ok ? fast_exp2(s2 - m_new) : 0.f;
@@ -445,26 +448,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_decode_kernel(const __grid_con
                         const int ts = lane / C::VAL;
                         // interleave token sub-lanes so that the two half-warps read disjoint banks
                         const int tsub = C::VTL == 4 ? ((ts & 1) * 2 + (ts >> 1)) : ts;
-#pragma unroll 4
-                        for (int j0 = 0; j0 < 32; j0 += C::VTL) {
-                            const int j = j0 + tsub;
-                            const float pb = __shfl_sync(0xffffffffu, pj, j);
-                            if (j < nv) {
-                                const uint2 u = *reinterpret_cast<const uint2*>(
-                                    st + size_t(srow0 + j) * (C::ROW * 2) + (C::RK + 4 * al) * 2);
-                                acc[hw][0] = fmaf(pb, bf16_lo(u.x), acc[hw][0]);
-                                acc[hw][1] = fmaf(pb, bf16_hi(u.x), acc[hw][1]);
-                                acc[hw][2] = fmaf(pb, bf16_lo(u.y), acc[hw][2]);
-                                acc[hw][3] = fmaf(pb, bf16_hi(u.y), acc[hw][3]);
+                        const uint8_t* vb = st + size_t(srow0 + tsub) * (C::ROW * 2) + (C::RK + 4 * al) * 2;
+                        float a0v = 0.f, a1v = 0.f, a2v = 0.f, a3v = 0.f;
+                        if (nv == 32) {
+#pragma unroll
+                            for (int j0 = 0; j0 < 32; j0 += C::VTL) {
+                                const float pb = __shfl_sync(0xffffffffu, pj, j0 + tsub);
+                                const uint2 u = *reinterpret_cast<const uint2*>(vb + j0 * (C::ROW * 2));
+                                a0v = fmaf(pb, bf16_lo(u.x), a0v);
+                                a1v = fmaf(pb, bf16_hi(u.x), a1v);
+                                a2v = fmaf(pb, bf16_lo(u.y), a2v);
+                                a3v = fmaf(pb, bf16_hi(u.y), a3v);
+                            }
+                        } else {
+                            // rows past the context may hold any bits: their p is 0 but 0 * NaN is
+                            // not, so they are skipped rather than weighted
+                            for (int j0 = 0; j0 < 32; j0 += C::VTL) {
+                                const float pb = __shfl_sync(0xffffffffu, pj, j0 + tsub);
+                                if (j0 + tsub < nv) {
+                                    const uint2 u = *reinterpret_cast<const uint2*>(vb + j0 * (C::ROW * 2));
+                                    a0v = fmaf(pb, bf16_lo(u.x), a0v);
+                                    a1v = fmaf(pb, bf16_hi(u.x), a1v);
+                                    a2v = fmaf(pb, bf16_lo(u.y), a2v);
+                                    a3v = fmaf(pb, bf16_hi(u.y), a3v);
+                                }
                             }
                         }
+                        acc[hw][0] += a0v;
+                        acc[hw][1] += a1v;
+                        acc[hw][2] += a2v;
+                        acc[hw][3] += a3v;
                     } else {
+                        const uint16_t* vr0 =
+                            reinterpret_cast<const uint16_t*>(st + size_t(srow0) * (C::ROW * 2) + C::RK * 2) + lane;
                         for (int j = 0; j < nv; ++j) {
                             const float pb = __shfl_sync(0xffffffffu, pj, j);
-                            const uint16_t* vr = reinterpret_cast<const uint16_t*>(
-                                st + size_t(srow0 + j) * (C::ROW * 2) + C::RK * 2);
+                            const uint16_t* vr = vr0 + j * C::ROW;
 #pragma unroll
-                            for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[lane + 32 * v]), acc[hw][v]);
+                            for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[32 * v]), acc[hw][v]);
                         }
                     }
                     __syncwarp();
@@ -511,6 +532,7 @@ struct ProParams {
     float scale;
 };
 
+template <class C>
 __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
     // every block helps initialise the split records to "empty" (m = -inf, l = 0)
     {
@@ -557,73 +579,97 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         if (threadIdx.x == 0) p.P[p.B] = carry;
         return;
     }
-    // (b, h) block: M_q image rows of head h
-    const int bh = blockIdx.x - 1;
-    if (bh >= p.B * p.H) return;
-    const int b = bh / p.H, h = bh % p.H;
-    const int DH = p.DH, half = DH / 2, RK = p.RK;
-    __shared__ float qr[256];
+    // (head, 16 sequences) block: this head's rows of the M_q images of those sequences
+    constexpr int DH = C::DH, RK = C::RK, half = DH / 2, KC = DH / 8;
+    constexpr int ITEMS = ((RK + 1) * KC + 255) / 256;  // (row, 8-wide k chunk) items per thread
+    const int blk = blockIdx.x - 1;
+    const int h = blk % C::H, b0 = (blk / C::H) * kProSeqs;
+    extern __shared__ __align__(16) float wt[];  // [(RK + 1) * DH]: [n][i], W^K_up,t column n (n == RK: mu)
+    __shared__ __align__(16) float qr[DH];
     __shared__ float red[8];
-    int qp = p.q_pos[b];
-    if (qp < 0 || qp >= p.max_pos) {
-        qp = qp < 0 ? 0 : p.max_pos - 1;
-        if (h == 0 && threadIdx.x == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
-    }
-    const float* qv = p.q + (size_t(b) * p.H + h) * DH;
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const float c = p.rope_cos[size_t(qp) * half + i], s = p.rope_sin[size_t(qp) * half + i];
-        const float lo = qv[i], hi = qv[i + half];
-        qr[i] = p.scale * (lo * c - hi * s);
-        qr[i + half] = p.scale * (hi * c + lo * s);
-    }
-    __syncthreads();
     size_t w_off, mu_off;
     if (p.variant == 0) {
-        w_off = ((size_t(p.layer) * p.H + h) * p.T + p.loop) * size_t(DH) * RK;
-        mu_off = (size_t(p.layer) * p.H + h) * size_t(p.T) * DH + size_t(p.loop) * DH;
+        w_off = ((size_t(p.layer) * C::H + h) * p.T + p.loop) * size_t(DH) * RK;
+        mu_off = (size_t(p.layer) * C::H + h) * size_t(p.T) * DH + size_t(p.loop) * DH;
     } else {
-        w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(DH) * RK;
-        mu_off = size_t(p.layer) * p.T * p.H * DH + (size_t(p.loop) * p.H + h) * DH;
+        w_off = ((size_t(p.layer) * p.T + p.loop) * C::H + h) * size_t(DH) * RK;
+        mu_off = size_t(p.layer) * p.T * C::H * DH + (size_t(p.loop) * C::H + h) * DH;
     }
-    const float* W = p.w_up_k + w_off;
-    const float* mu = p.mu_k + mu_off;
-    // element (n, k) of this head's block of M_q^T: n < RK latent column, n == RK bias
-    auto value = [&](int n, int k) -> float {
-        const int i = k < half ? k : k - half;
-        const float wl = n < RK ? W[size_t(i) * RK + n] : mu[i];
-        const float wh = n < RK ? W[size_t(i + half) * RK + n] : mu[i + half];
-        return k < half ? qr[i] * wl + qr[i + half] * wh : qr[i + half] * wl - qr[i] * wh;
-    };
-    float mx = 0.f;
-    for (int e = threadIdx.x; e < (RK + 1) * DH; e += blockDim.x) mx = fmaxf(mx, fabsf(value(e / DH, e % DH)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    mx = 0.f;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) mx = fmaxf(mx, red[i]);
-    // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
-    int e2 = 0;
-    float scale = 1.f;
-    if (mx > 0.f && isfinite(mx)) {
-        frexpf(mx, &e2);  // mx < 2^e2
-        scale = ldexpf(1.f, 15 - e2);
+    for (int e = threadIdx.x; e < DH * RK; e += blockDim.x) {
+        const int i = e / RK, n = e % RK;
+        wt[n * DH + i] = p.w_up_k[w_off + e];
     }
-    const int part = h / p.HC, hc = h % p.HC, g = hc / p.HG, hg = hc % p.HG;
-    uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(p.GPC) * p.NG * DH * 2 + size_t(g) * p.NG * DH * 2;
-    for (int e = threadIdx.x; e < (RK + 1) * DH; e += blockDim.x) {
-        const int n = e / DH, k = e % DH;
-        const int rowi = n < RK ? hg * RK + n : p.HG * RK + hg;
-        const __half v = __float2half_rn(value(n, k) * scale);
-        *reinterpret_cast<__half*>(img + sm100::sw128_offset(rowi, k, p.NG)) = v;
-    }
-    if (hg == 0) {  // zero the group's padding rows
-        for (int e = threadIdx.x; e < (p.NG - p.HG * (RK + 1)) * DH; e += blockDim.x) {
-            const int rowi = p.HG * (RK + 1) + e / DH, k = e % DH;
-            *reinterpret_cast<__half*>(img + sm100::sw128_offset(rowi, k, p.NG)) = __float2half_rn(0.f);
+    for (int i = threadIdx.x; i < DH; i += blockDim.x) wt[RK * DH + i] = p.mu_k[mu_off + i];
+    const int part = h / C::HC, hc = h % C::HC, g = hc / C::HG, hg = hc % C::HG;
+    for (int b = b0; b < min(p.B, b0 + kProSeqs); ++b) {
+        int qp = p.q_pos[b];
+        if (qp < 0 || qp >= p.max_pos) {
+            qp = qp < 0 ? 0 : p.max_pos - 1;
+            if (h == 0 && threadIdx.x == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
         }
+        __syncthreads();  // wt ready; previous sequence done with qr / red
+        const float* qv = p.q + (size_t(b) * C::H + h) * DH;
+        for (int i = threadIdx.x; i < half; i += blockDim.x) {
+            const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
+            const float lo = qv[i], hi = qv[i + half];
+            qr[i] = p.scale * (lo * c - hi * sn);
+            qr[i + half] = p.scale * (hi * c + lo * sn);
+        }
+        __syncthreads();
+        // element (n, k): k < d/2: q'_k w_k + q'_{k+d/2} w_{k+d/2};  k >= d/2: q'_{i+d/2} w_i - q'_i w_{i+d/2}
+        float val[ITEMS][8];
+        float mx = 0.f;
+#pragma unroll
+        for (int it = 0; it < ITEMS; ++it) {
+            const int e = threadIdx.x + it * 256;
+            if (e < (RK + 1) * KC) {
+                const int n = e / KC, k0 = (e % KC) * 8;
+                const int i0 = k0 < half ? k0 : k0 - half;
+                const float* wn = wt + n * DH;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + u;
+                    const float wl = wn[i], wh = wn[i + half], ql = qr[i], qh = qr[i + half];
+                    val[it][u] = k0 < half ? ql * wl + qh * wh : qh * wl - ql * wh;
+                    mx = fmaxf(mx, fabsf(val[it][u]));
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red[i]);
+        // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
+        int e2 = 0;
+        float scale = 1.f;
+        if (mx > 0.f && isfinite(mx)) {
+            frexpf(mx, &e2);  // mx < 2^e2
+            scale = ldexpf(1.f, 15 - e2);
+        }
+        uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
+#pragma unroll
+        for (int it = 0; it < ITEMS; ++it) {
+            const int e = threadIdx.x + it * 256;
+            if (e < (RK + 1) * KC) {
+                const int n = e / KC, k0 = (e % KC) * 8;
+                const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
+                __align__(16) __half v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = __float2half_rn(val[it][u] * scale);
+                *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) =
+                    *reinterpret_cast<const uint4*>(v);
+            }
+        }
+        if (hg == 0)  // the group's padding rows
+            for (int e = threadIdx.x; e < (C::NG - C::HG * (RK + 1)) * KC; e += blockDim.x) {
+                const int rowi = C::HG * (RK + 1) + e / KC, k0 = (e % KC) * 8;
+                *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = make_uint4(0, 0, 0, 0);
+            }
+        if (threadIdx.x == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
     }
-    if (threadIdx.x == 0) p.inv_scale[size_t(b) * p.H + h] = kLog2e / scale;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -715,7 +761,9 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.loop = call.loop;
     pp.variant = c->desc.variant;
     pp.scale = call.scale;
-    tc_prologue_kernel<<<1 + B * C::H, 256, 0, call.stream>>>(pp);
+    const int pro_smem = (C::RK + 1) * C::DH * int(sizeof(float));
+    LLA_CUDA_TRY(cudaFuncSetAttribute(tc_prologue_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, pro_smem));
+    tc_prologue_kernel<C><<<1 + C::H * ((B + kProSeqs - 1) / kProSeqs), 256, pro_smem, call.stream>>>(pp);
     LLA_CUDA_TRY(cudaGetLastError());
 
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).
@@ -744,7 +792,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tp.G = G;
     LLA_CUDA_TRY(cudaFuncSetAttribute(tc_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     if (call.ev_begin) LLA_CUDA_TRY(cudaEventRecord(call.ev_begin, call.stream));
-    tc_decode_kernel<C><<<G, kThreads, C::SMEM, call.stream>>>(map, tp);
+    tc_decode_kernel<C><<<G, C::THREADS, C::SMEM, call.stream>>>(map, tp);
     LLA_CUDA_TRY(cudaGetLastError());
     if (call.ev_end) LLA_CUDA_TRY(cudaEventRecord(call.ev_end, call.stream));
     lla_tc_ranges ranges;
