@@ -113,6 +113,19 @@ lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int l
                              const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
                              int max_tokens, cudaStream_t stream) {
     const lla_codec_desc& ds = c->desc;
+    // the tensor-core kernel where it applies (TMA needs 16-byte aligned rows and stacks)
+    if ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(store) & 15) == 0) {
+        const lla_status st =
+            lla_encode_tc(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+        if (st != LLA_ERR_UNSUPPORTED_SHAPE) return st;
+    }
+    return lla_encode_simt(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+}
+
+lla_status lla_encode_simt(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                           const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
+                           int max_tokens, cudaStream_t stream) {
+    const lla_codec_desc& ds = c->desc;
     if (ds.r_k > kMaxR || ds.r_v > kMaxR) return LLA_ERR_UNSUPPORTED_SHAPE;
     EncodeParams p;
     p.x = x;

@@ -1,0 +1,337 @@
+// Tensor-core LLA encode: c = (x - mu) W_down = x W_down - b  [LLA §3 eq. (2)].
+//
+// One CTA per (128-token tile, layer, head): the loop stacks x of the tile
+// (K axis and V axis, S = T*d_head each, or T*H*d_head for LLA-2D) are the A
+// operand and W_down^T of the two axes the B operands of tcgen05.mma
+// (bf16 in, fp32 accumulators in TMEM: r_k columns for K, r_v for V).  K is
+// walked in 64-element chunks staged by TMA with the 128-byte swizzle into a
+// ring of shared-memory stages.  Four epilogue warps (thread = token row)
+// subtract b = mu W_down, round to bf16 (nearest-even) and write the token's
+// K || V latent row to the store slot (seq_idx[i], tok_idx[i]).
+//
+//   warp 0  TMA producer        warp 1  TMEM allocator + MMA issuer
+//   warps 2-5  epilogue
+// Waits are bounded (sm100.cuh); a wait that gives up sets a bit in the
+// codec's status word and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "lla_internal.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTok = 128;
+constexpr int kKc = 64;  // K elements per stage (one 128-byte swizzle atom)
+constexpr int kThreads = 192;
+constexpr int kSmemLimit = 232448;
+
+constexpr int pow2_at_least(int x) {
+    int p = 32;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+template <int RK_, int RV_>
+struct ECfg {
+    static constexpr int RK = RK_, RV = RV_;
+    static constexpr int A_BYTES = kTok * kKc * 2;  // one axis' stacks of the 128 tokens, 64 K elements
+    static constexpr int BK_BYTES = RK * kKc * 2;
+    static constexpr int BV_BYTES = RV * kKc * 2;
+    static constexpr int STAGE = 2 * A_BYTES + BK_BYTES + BV_BYTES;  // [A_K | A_V | W_K | W_V]
+    // two CTAs per SM when two stages fit in half the shared memory, else one CTA with up to 4 stages
+    static constexpr int NST2 = (kSmemLimit / 2 - 2048) / STAGE;
+    static constexpr int NST1 = (kSmemLimit - 2048) / STAGE;
+    static constexpr int NST = NST2 >= 2 ? (NST2 > 4 ? 4 : NST2) : (NST1 > 4 ? 4 : NST1);
+    static constexpr int SMEM = 1024 + NST * STAGE + 1024;
+    static constexpr int VCOL = (RK + 31) / 32 * 32;  // TMEM column of the V accumulator
+    static constexpr int TMEM_COLS = pow2_at_least(VCOL + RV);
+    static constexpr uint32_t IDESC_K = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(RK >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+    static constexpr uint32_t IDESC_V = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(RV >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+    static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= 256 && RV <= 256, "ranks");
+    static_assert(TMEM_COLS <= 512, "TMEM");
+    static_assert(SMEM <= kSmemLimit, "shared memory");
+};
+
+struct EncParams {
+    const int32_t* seq_idx;
+    const int32_t* tok_idx;
+    uint16_t* store;
+    const float* bias_k;  // [D][Hg][r_k]
+    const float* bias_v;
+    uint32_t* status;
+    int n, layer_begin, num_layers, Hg, S, D, batch, max_tokens;
+    size_t row;  // elements per (sequence, layer, token) row of the store
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // x = lo, y = hi
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <class C>
+__global__ void __launch_bounds__(kThreads) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                              const __grid_constant__ CUtensorMap wkmap,
+                                                              const __grid_constant__ CUtensorMap wvmap,
+                                                              EncParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NST * C::STAGE);
+    uint64_t* full = bars;                 // [NST]
+    uint64_t* empty = bars + C::NST;       // [NST]
+    uint64_t* acc_full = bars + 2 * C::NST;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x;
+    const int slot = blockIdx.y;  // L * Hg + h
+    const int L = slot / p.Hg, h = slot - L * p.Hg;
+    const int layer = p.layer_begin + L;
+    const int nk = p.S / kKc;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NST; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, 1);
+        }
+        mbar_init(acc_full, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (elect_one()) {
+            prefetch_tensormap(&xmap);
+            prefetch_tensormap(&wkmap);
+            prefetch_tensormap(&wvmap);
+            const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
+            const int wrow_k = (layer * p.Hg + h) * C::RK, wrow_v = (layer * p.Hg + h) * C::RV;
+            int issued = 0;
+            for (int kc = 0; kc < nk; ++kc) {
+                const int s = kc % C::NST, round = kc / C::NST;
+                if (round > 0 && !mbar_wait(empty + s, (round - 1) & 1, p.status, 4u, 20)) break;
+                uint8_t* st = smem + size_t(s) * C::STAGE;
+                mbar_expect_tx(full + s, C::STAGE);
+                // x: dims (S, slot = (L*Hg + h)*2 + axis, token): one box per axis
+                for (int axis = 0; axis < 2; ++axis)
+                    asm volatile(
+                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st + axis * C::A_BYTES)),
+                        "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(kc * kKc), "r"(slot * 2 + axis), "r"(tile * kTok),
+                        "r"(smem_u32(full + s)), "l"(pol_x)
+                        : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                    " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES)),
+                    "l"(reinterpret_cast<uint64_t>(&wkmap)), "r"(kc * kKc), "r"(wrow_k), "r"(smem_u32(full + s)),
+                    "l"(pol_w)
+                    : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                    " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES + C::BK_BYTES)),
+                    "l"(reinterpret_cast<uint64_t>(&wvmap)), "r"(kc * kKc), "r"(wrow_v), "r"(smem_u32(full + s)),
+                    "l"(pol_w)
+                    : "memory");
+                ++issued;
+            }
+            // drain: no copy in flight at exit
+            for (int s = 0; s < C::NST && s < issued; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % C::NST);
+                mbar_wait(full + s, (last / C::NST) & 1, p.status, 4u, 21);
+            }
+        }
+    } else if (warp == 1) {
+        if (elect_one()) {
+            bool ok = true;
+            for (int kc = 0; kc < nk && ok; ++kc) {
+                const int s = kc % C::NST, round = kc / C::NST;
+                if (!(ok = mbar_wait(full + s, round & 1, p.status, 4u, 22))) break;
+                tc_fence_after();
+                const uint32_t ak = smem_u32(smem + size_t(s) * C::STAGE), av = ak + C::A_BYTES;
+                const uint32_t bk = av + C::A_BYTES, bv = bk + C::BK_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < kKc / 16; ++kk) {
+                    const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+                    mma_f16_ss(tmem, sw128_kmajor_desc(ak + kk * 32), sw128_kmajor_desc(bk + kk * 32), C::IDESC_K, acc);
+                    mma_f16_ss(tmem + C::VCOL, sw128_kmajor_desc(av + kk * 32), sw128_kmajor_desc(bv + kk * 32),
+                               C::IDESC_V, acc);
+                }
+                mma_commit(empty + s);
+            }
+            mma_commit(acc_full);
+            mbar_wait(acc_full, 0, p.status, 4u, 23);
+        }
+    } else {
+        // epilogue: warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+        const int qd = warp & 3;
+        const int r = 32 * qd + lane;
+        const int i = tile * kTok + r;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.status, 4u, 24));
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(32 * qd) << 16);
+        int sq = -1, tk = -1;
+        if (i < p.n) {
+            sq = p.seq_idx[i];
+            tk = p.tok_idx[i];
+        }
+        const bool write = ok && i < p.n && sq >= 0 && sq < p.batch && tk >= 0 && tk < p.max_tokens;
+        uint16_t* dst = p.store + ((size_t(sq < 0 ? 0 : sq) * p.D + layer) * p.max_tokens + (tk < 0 ? 0 : tk)) * p.row +
+                        size_t(h) * (C::RK + C::RV);
+        const float* bk = p.bias_k + (size_t(layer) * p.Hg + h) * C::RK;
+        const float* bv = p.bias_v + (size_t(layer) * p.Hg + h) * C::RV;
+#pragma unroll
+        for (int a0 = 0; a0 < C::RK; a0 += 16) {
+            float v[16];
+            tmem_ld<16>(taddr + a0, v);
+            tmem_wait_ld();
+            if (write) {
+                uint4 w0, w1;
+                w0.x = pack_bf16(v[0] - bk[a0 + 0], v[1] - bk[a0 + 1]);
+                w0.y = pack_bf16(v[2] - bk[a0 + 2], v[3] - bk[a0 + 3]);
+                w0.z = pack_bf16(v[4] - bk[a0 + 4], v[5] - bk[a0 + 5]);
+                w0.w = pack_bf16(v[6] - bk[a0 + 6], v[7] - bk[a0 + 7]);
+                w1.x = pack_bf16(v[8] - bk[a0 + 8], v[9] - bk[a0 + 9]);
+                w1.y = pack_bf16(v[10] - bk[a0 + 10], v[11] - bk[a0 + 11]);
+                w1.z = pack_bf16(v[12] - bk[a0 + 12], v[13] - bk[a0 + 13]);
+                w1.w = pack_bf16(v[14] - bk[a0 + 14], v[15] - bk[a0 + 15]);
+                reinterpret_cast<uint4*>(dst + a0)[0] = w0;
+                reinterpret_cast<uint4*>(dst + a0)[1] = w1;
+            }
+        }
+#pragma unroll
+        for (int a0 = 0; a0 < C::RV; a0 += 16) {
+            float v[16];
+            tmem_ld<16>(taddr + C::VCOL + a0, v);
+            tmem_wait_ld();
+            if (write) {
+                uint4 w0, w1;
+                w0.x = pack_bf16(v[0] - bv[a0 + 0], v[1] - bv[a0 + 1]);
+                w0.y = pack_bf16(v[2] - bv[a0 + 2], v[3] - bv[a0 + 3]);
+                w0.z = pack_bf16(v[4] - bv[a0 + 4], v[5] - bv[a0 + 5]);
+                w0.w = pack_bf16(v[6] - bv[a0 + 6], v[7] - bv[a0 + 7]);
+                w1.x = pack_bf16(v[8] - bv[a0 + 8], v[9] - bv[a0 + 9]);
+                w1.y = pack_bf16(v[10] - bv[a0 + 10], v[11] - bv[a0 + 11]);
+                w1.z = pack_bf16(v[12] - bv[a0 + 12], v[13] - bv[a0 + 13]);
+                w1.w = pack_bf16(v[14] - bv[a0 + 14], v[15] - bv[a0 + 15]);
+                reinterpret_cast<uint4*>(dst + C::RK + a0)[0] = w0;
+                reinterpret_cast<uint4*>(dst + C::RK + a0)[1] = w1;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+bool make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+    cuuint32_t es[3] = {1u, 1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class C>
+lla_status run_encode(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                      const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
+                      cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return LLA_ERR_CUDA;
+    const lla_codec_desc& ds = c->desc;
+    const int Hg = ds.variant == 0 ? ds.H : 1;
+    const int S = c->S;
+    CUtensorMap xmap, wkmap, wvmap;
+    {
+        cuuint64_t dims[3] = {cuuint64_t(S), cuuint64_t(num_layers) * Hg * 2, cuuint64_t(n)};
+        cuuint64_t strides[2] = {cuuint64_t(S) * 2, cuuint64_t(num_layers) * Hg * 2 * S * 2};
+        cuuint32_t box[3] = {uint32_t(kKc), 1u, uint32_t(kTok)};
+        if (!make_map(enc, &xmap, x, 3, dims, strides, box)) return LLA_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {cuuint64_t(S), cuuint64_t(ds.D) * Hg * C::RK};
+        cuuint64_t strides[1] = {cuuint64_t(S) * 2};
+        cuuint32_t box[2] = {uint32_t(kKc), uint32_t(C::RK)};
+        if (!make_map(enc, &wkmap, c->w_down_k_t, 2, dims, strides, box)) return LLA_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {cuuint64_t(S), cuuint64_t(ds.D) * Hg * C::RV};
+        cuuint64_t strides[1] = {cuuint64_t(S) * 2};
+        cuuint32_t box[2] = {uint32_t(kKc), uint32_t(C::RV)};
+        if (!make_map(enc, &wvmap, c->w_down_v_t, 2, dims, strides, box)) return LLA_ERR_CUDA;
+    }
+    EncParams p;
+    p.seq_idx = seq_idx;
+    p.tok_idx = tok_idx;
+    p.store = store;
+    p.bias_k = c->bias_k;
+    p.bias_v = c->bias_v;
+    p.status = c->status;
+    p.n = n;
+    p.layer_begin = layer_begin;
+    p.num_layers = num_layers;
+    p.Hg = Hg;
+    p.S = S;
+    p.D = ds.D;
+    p.batch = batch;
+    p.max_tokens = max_tokens;
+    p.row = size_t(ds.r_k + ds.r_v) * Hg;
+    LLA_CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    dim3 grid((n + kTok - 1) / kTok, num_layers * Hg);
+    encode_tc_kernel<C><<<grid, kThreads, C::SMEM, stream>>>(xmap, wkmap, wvmap, p);
+    LLA_CUDA_TRY(cudaGetLastError());
+    return LLA_OK;
+}
+
+}  // namespace
+
+// Tensor-core encode for the codec shapes it is built for; LLA_ERR_UNSUPPORTED_SHAPE otherwise.
+lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                         const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
+                         cudaStream_t stream) {
+    const lla_codec_desc& d = c->desc;
+    if (c->S % kKc != 0 || !c->status) return LLA_ERR_UNSUPPORTED_SHAPE;
+    if (d.r_k == 16 && d.r_v == 32)
+        return run_encode<ECfg<16, 32>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+    if (d.r_k == 96 && d.r_v == 160)
+        return run_encode<ECfg<96, 160>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+    if (d.r_k == 64 && d.r_v == 128)
+        return run_encode<ECfg<64, 128>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+    return LLA_ERR_UNSUPPORTED_SHAPE;
+}

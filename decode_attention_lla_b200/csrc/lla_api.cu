@@ -54,7 +54,7 @@ lla_status dev_alloc(T** p, size_t count) {
 void codec_free(lla_codec* c) {
     if (!c) return;
     void* ptrs[] = {c->w_up_k, c->w_up_v, c->mu_k, c->mu_v, c->bias_k, c->bias_v,
-                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles};
+                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles, c->status};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete c;
@@ -119,7 +119,8 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
         (st = dev_alloc(&c->mu_k, nmu)) || (st = dev_alloc(&c->mu_v, nmu)) ||
         (st = dev_alloc(&c->bias_k, groups * rk)) || (st = dev_alloc(&c->bias_v, groups * rv)) ||
         (st = dev_alloc(&c->w_down_k_t, groups * rk * S)) || (st = dev_alloc(&c->w_down_v_t, groups * rv * S)) ||
-        (st = dev_alloc(&c->rope_cos, nrope)) || (st = dev_alloc(&c->rope_sin, nrope))) {
+        (st = dev_alloc(&c->rope_cos, nrope)) || (st = dev_alloc(&c->rope_sin, nrope)) ||
+        (st = dev_alloc(&c->status, 4))) {
         codec_free(c);
         return st;
     }
@@ -163,7 +164,8 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
               cudaMemcpyAsync(c->w_down_k_t, wdt_k.data(), wdt_k.size() * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->w_down_v_t, wdt_v.data(), wdt_v.size() * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->rope_cos, rc.data(), rc.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
-              cudaMemcpyAsync(c->rope_sin, rs.data(), rs.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+              cudaMemcpyAsync(c->rope_sin, rs.data(), rs.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemsetAsync(c->status, 0, 4 * sizeof(uint32_t), stream) == cudaSuccess;
     if (ok) ok = lla_build_phi_tiles(c, stream) == LLA_OK;
     if (ok) ok = cudaStreamSynchronize(stream) == cudaSuccess;
     if (!ok) {

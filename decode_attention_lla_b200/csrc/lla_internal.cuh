@@ -29,6 +29,9 @@ struct lla_codec {
     // image the tensor-core decode kernel feeds to tcgen05.mma.
     uint16_t* phi_tiles = nullptr;
     int phi_num_tiles = 0;
+    // Device status words of the tensor-core encode (bit 2: a bounded wait gave up; word 1:
+    // the first wait site that did).
+    uint32_t* status = nullptr;
 };
 
 // Workspace header (first 256 bytes of every decode workspace).
@@ -88,6 +91,12 @@ lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int l
                              int num_layers, const int32_t* seq_idx, const int32_t* tok_idx,
                              uint16_t* store, int batch, int max_tokens, cudaStream_t stream);
 lla_status lla_build_phi_tiles(lla_codec* c, cudaStream_t stream);
+lla_status lla_encode_simt(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                           const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
+                           int max_tokens, cudaStream_t stream);
+lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                         const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
+                         cudaStream_t stream);
 
 int lla_num_sms();
 
