@@ -8,17 +8,17 @@
 // which equals sum_j p_j v_hat_j because the normalised p_j sum to one
 // [LLA §3 eq. (3)].  An empty context (no records with l > 0) yields zeros.
 //
-// One CTA per (head, group of sequences): W^V_up,t of the head is staged in
-// shared memory once, transposed so that the threads of a warp (one output
-// dimension each) read consecutive words.
+// One CTA per (head, 16 sequences), one warp per sequence: W^V_up,t of the head
+// is staged in shared memory once, transposed so that the lanes of a warp (one
+// output dimension each) read consecutive words.
 #include <math.h>
 
 #include "lla_internal.cuh"
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kSeqPerCta = 16;
+constexpr int kThreads = 512;
+constexpr int kSeqPerCta = kThreads / 32;  // one warp per sequence
 
 struct CombineParams {
     const float* partials;
@@ -66,15 +66,16 @@ __device__ __forceinline__ void record_range(const CombineParams& p, int b, int 
     }
 }
 
+// One warp per (sequence, head); the CTA's sixteen warps share W^V_up,t of one head.
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     const int h = blockIdx.x;
-    const int b0 = blockIdx.y * kSeqPerCta;
-    const int tid = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y * kSeqPerCta + warp;
     const int d = p.d, rv = p.r_v;
     extern __shared__ float smem[];
-    float* Wt = smem;           // [rv][d]
-    float* mu = Wt + rv * d;    // [d]
-    float* abar = mu + d;       // [rv]
+    float* Wt = smem;                     // [rv][d]
+    float* mu = Wt + rv * d;              // [d]
+    float* abar = mu + d + warp * rv;     // [kSeqPerCta][rv]
 
     size_t w_off, mu_off;
     if (p.variant == 0) {
@@ -84,47 +85,68 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
         w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(d) * rv;
         mu_off = size_t(p.layer) * p.T * p.H * d + (size_t(p.loop) * p.H + h) * d;
     }
-    for (int idx = tid; idx < d * rv; idx += kThreads) {
-        const int i = idx / rv, a = idx - i * rv;
-        Wt[a * d + i] = p.w_up_v[w_off + idx];
+    // transposed into shared memory: consecutive threads write consecutive i (no bank conflicts)
+    for (int idx = threadIdx.x; idx < d * rv; idx += blockDim.x) {
+        const int a = idx / d, i = idx - a * d;
+        Wt[idx] = __ldg(p.w_up_v + w_off + size_t(i) * rv + a);
     }
-    for (int i = tid; i < d; i += kThreads) mu[i] = p.mu_v[mu_off + i];
+    for (int i = threadIdx.x; i < d; i += blockDim.x) mu[i] = __ldg(p.mu_v + mu_off + i);
     __syncthreads();
+    if (b >= p.B) return;
 
     const size_t rec_len = lla_partial_floats(rv);
-    for (int b = b0; b < min(p.B, b0 + kSeqPerCta); ++b) {
-        int s0, s1, hr, hs;
-        record_range(p, b, h, s0, s1, hr, hs);
-        float M = -INFINITY;
-        for (int s = s0; s < s1; ++s) M = fmaxf(M, p.partials[(size_t(s) * hs + hr) * rec_len]);
-        float L = 0.f;
-        if (M != -INFINITY)
-            for (int s = s0; s < s1; ++s) {
-                const float* rec = p.partials + (size_t(s) * hs + hr) * rec_len;
-                if (rec[0] != -INFINITY) L += rec[1] * expf(rec[0] - M);
-            }
-        for (int a = tid; a < rv; a += kThreads) {
-            float v = 0.f;
-            if (L > 0.f) {
-                for (int s = s0; s < s1; ++s) {
-                    const float* rec = p.partials + (size_t(s) * hs + hr) * rec_len;
-                    if (rec[0] != -INFINITY) v += rec[2 + a] * expf(rec[0] - M);
-                }
-                v /= L;
-            }
-            abar[a] = v;
+    int s0, s1, hr, hs;
+    record_range(p, b, h, s0, s1, hr, hs);
+    auto rec = [&](int s) { return p.partials + (size_t(s) * hs + hr) * rec_len; };
+    // merged maximum and normaliser over the records (log-sum-exp); a record with l = 0
+    // saw no valid token and is skipped whatever its m holds
+    float M = -INFINITY;
+    for (int s = s0 + lane; s < s1; s += 32) {
+        const float* r = rec(s);
+        if (r[1] > 0.f) M = fmaxf(M, r[0]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    if (M != -INFINITY)
+        for (int s = s0 + lane; s < s1; s += 32) {
+            const float* r = rec(s);
+            if (r[1] > 0.f) L += r[1] * expf(r[0] - M);
         }
-        __syncthreads();
-        float* o = p.out + (size_t(b) * p.H + h) * d;
-        for (int i = tid; i < d; i += kThreads) {
-            float v = 0.f;
-            if (L > 0.f) {
-                v = mu[i];
-                for (int a = 0; a < rv; ++a) v = fmaf(abar[a], Wt[a * d + i], v);
-            }
-            o[i] = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float* o = p.out + (size_t(b) * p.H + h) * d;
+    if (!(L > 0.f)) {  // empty context
+        for (int i = lane; i < d; i += 32) o[i] = 0.f;
+        return;
+    }
+    // record weights exp(m_s - M) / L, one per lane, broadcast by shuffle
+    const float invL = 1.f / L;
+    for (int a = lane; a < rv; a += 32) abar[a] = 0.f;
+    for (int sb = s0; sb < s1; sb += 32) {
+        float wgt = 0.f;
+        if (sb + lane < s1) {
+            const float* r = rec(sb + lane);
+            if (r[1] > 0.f) wgt = expf(r[0] - M) * invL;
         }
-        __syncthreads();
+        const int ns = min(32, s1 - sb);
+        for (int a0 = 0; a0 < rv; a0 += 32) {  // whole warp in every iteration (shuffles)
+            const int a = a0 + lane;
+            float v = a < rv ? abar[a] : 0.f;
+#pragma unroll 4
+            for (int j = 0; j < ns; ++j) {
+                const float wj = __shfl_sync(0xffffffffu, wgt, j);
+                if (wj != 0.f && a < rv) v = fmaf(rec(sb + j)[2 + a], wj, v);
+            }
+            if (a < rv) abar[a] = v;
+        }
+    }
+    __syncwarp();
+    // out = abar W^V_up,t^T + mu^V_t
+    for (int i = lane; i < d; i += 32) {
+        float v = mu[i];
+        for (int a = 0; a < rv; ++a) v = fmaf(abar[a], Wt[a * d + i], v);
+        o[i] = v;
     }
 }
 
@@ -168,7 +190,7 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     p.layer = call.layer;
     p.loop = call.loop;
     p.variant = ds.variant;
-    const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + ds.r_v) * sizeof(float);
+    const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     dim3 grid(ds.H, (call.batch + kSeqPerCta - 1) / kSeqPerCta);
     combine_kernel<<<grid, kThreads, smem, call.stream>>>(p);

@@ -51,7 +51,6 @@ constexpr int kMaxCtas = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kFlagTimeout = 4u;
-constexpr int kProSeqs = 16;  // sequences per prologue block
 
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
@@ -85,7 +84,9 @@ struct Cfg {
     static constexpr int THREADS = 32 * (2 + NCW);
     static constexpr int HPW = HC / WPQ;  // heads per compute warp
     static constexpr int TMEM_COLS = 512;
-    static constexpr int BUF_COLS = 256;
+    // TMEM accumulator ring: as many NG-column buffers as fit in 512 columns (at most 4)
+    static constexpr int NBUF = (512 / NG) > 4 ? 4 : (512 / NG);
+    static constexpr int BUF_COLS = (512 / NBUF) / 16 * 16;
     static constexpr uint32_t IDESC = idesc_f16_f32(128, NG);
     // V-side lane mapping
     static constexpr bool VQUAD = (RV == 32 || RV == 64 || RV == 128);
@@ -184,9 +185,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     uint64_t* phi_empty = bars + 1;
     uint64_t* mq_full = bars + 2;
     uint64_t* mq_empty = bars + 3;
-    uint64_t* tm_full = bars + 4;   // [2]
-    uint64_t* tm_empty = bars + 6;  // [2]
-    uint64_t* st_full = bars + 8;   // [NST]
+    uint64_t* tm_full = bars + 4;            // [NBUF]
+    uint64_t* tm_empty = tm_full + C::NBUF;  // [NBUF]
+    uint64_t* st_full = tm_empty + C::NBUF;  // [NST]
     uint64_t* st_empty = st_full + C::NST;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(st_empty + C::NST);
     // issued[s] = number of loads the producer has issued into stage slot s.  Consumer warps
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         mbar_init(phi_empty, 1);
         mbar_init(mq_full, 1);
         mbar_init(mq_empty, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::NBUF; ++i) {
             mbar_init(tm_full + i, 1);
             mbar_init(tm_empty + i, C::NCW);
         }
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 ++phi_n;
                 tc_fence_after();
                 for (int g = 0; g < C::GPC && ok; ++g) {
-                    const uint32_t buf = gi & 1, use = gi >> 1;
+                    const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
                     if (use > 0 && !(ok = mbar_wait(tm_empty + buf, (use - 1) & 1, p.status, kFlagTimeout, 9))) break;
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + buf * C::BUF_COLS;
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
             const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this warp
 
             for (int g = 0; g < C::GPC && ok; ++g) {
-                const uint32_t buf = gi & 1, use = gi >> 1;
+                const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
                 ok = __all_sync(0xffffffffu, mbar_wait(tm_full + buf, use & 1, p.status, kFlagTimeout, 12));
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
@@ -420,20 +421,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
 
                     // ---- score: s = c^K . G + bias
-                    float sa = 0.f, sb = 0.f;
+                    // packed fp32 pairs: two latent dimensions per f32x2 FMA, two independent chains
+                    uint64_t s01 = 0, s23 = 0;
 #pragma unroll
                     for (int a0 = 0; a0 < C::RK; a0 += 8) {
                         const uint4 u = *reinterpret_cast<const uint4*>(myrow + a0 * 2);
-                        sa = fmaf(bf16_lo(u.x), gv[a0 + 0], sa);
-                        sb = fmaf(bf16_hi(u.x), gv[a0 + 1], sb);
-                        sa = fmaf(bf16_lo(u.y), gv[a0 + 2], sa);
-                        sb = fmaf(bf16_hi(u.y), gv[a0 + 3], sb);
-                        sa = fmaf(bf16_lo(u.z), gv[a0 + 4], sa);
-                        sb = fmaf(bf16_hi(u.z), gv[a0 + 5], sb);
-                        sa = fmaf(bf16_lo(u.w), gv[a0 + 6], sa);
-                        sb = fmaf(bf16_hi(u.w), gv[a0 + 7], sb);
+                        s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[a0 + 0], gv[a0 + 1]), s01);
+                        s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[a0 + 2], gv[a0 + 3]), s23);
+                        s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[a0 + 4], gv[a0 + 5]), s01);
+                        s23 = f2_fma(bf16x2_to_f2(u.w), f2_pack(gv[a0 + 6], gv[a0 + 7]), s23);
                     }
-                    const float s2 = row_ok ? (sa + sb + bias) * __ldg(isc_row + hl) : -INFINITY;
+                    const float2 sp = f2_unpack(s01), sq = f2_unpack(s23);
+                    const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * __ldg(isc_row + hl) : -INFINITY;
                     // ---- online softmax in base 2
                     const float m_new = fmaxf(m[hw], warp_max(s2));
                     const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m[hw] - m_new);
@@ -449,16 +448,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         // interleave token sub-lanes so that the two half-warps read disjoint banks
                         const int tsub = C::VTL == 4 ? ((ts & 1) * 2 + (ts >> 1)) : ts;
                         const uint8_t* vb = st + size_t(srow0 + tsub) * (C::ROW * 2) + (C::RK + 4 * al) * 2;
-                        float a0v = 0.f, a1v = 0.f, a2v = 0.f, a3v = 0.f;
+                        uint64_t v01 = 0, v23 = 0;  // packed fp32 pairs
                         if (nv == 32) {
 #pragma unroll
                             for (int j0 = 0; j0 < 32; j0 += C::VTL) {
                                 const float pb = __shfl_sync(0xffffffffu, pj, j0 + tsub);
                                 const uint2 u = *reinterpret_cast<const uint2*>(vb + j0 * (C::ROW * 2));
-                                a0v = fmaf(pb, bf16_lo(u.x), a0v);
-                                a1v = fmaf(pb, bf16_hi(u.x), a1v);
-                                a2v = fmaf(pb, bf16_lo(u.y), a2v);
-                                a3v = fmaf(pb, bf16_hi(u.y), a3v);
+                                const uint64_t pp = f2_pack(pb, pb);
+                                v01 = f2_fma(pp, bf16x2_to_f2(u.x), v01);
+                                v23 = f2_fma(pp, bf16x2_to_f2(u.y), v23);
                             }
                         } else {
                             // rows past the context may hold any bits: their p is 0 but 0 * NaN is
@@ -467,17 +465,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                                 const float pb = __shfl_sync(0xffffffffu, pj, j0 + tsub);
                                 if (j0 + tsub < nv) {
                                     const uint2 u = *reinterpret_cast<const uint2*>(vb + j0 * (C::ROW * 2));
-                                    a0v = fmaf(pb, bf16_lo(u.x), a0v);
-                                    a1v = fmaf(pb, bf16_hi(u.x), a1v);
-                                    a2v = fmaf(pb, bf16_lo(u.y), a2v);
-                                    a3v = fmaf(pb, bf16_hi(u.y), a3v);
+                                    const uint64_t pp = f2_pack(pb, pb);
+                                    v01 = f2_fma(pp, bf16x2_to_f2(u.x), v01);
+                                    v23 = f2_fma(pp, bf16x2_to_f2(u.y), v23);
                                 }
                             }
                         }
-                        acc[hw][0] += a0v;
-                        acc[hw][1] += a1v;
-                        acc[hw][2] += a2v;
-                        acc[hw][3] += a3v;
+                        const float2 w01 = f2_unpack(v01), w23 = f2_unpack(v23);
+                        acc[hw][0] += w01.x;
+                        acc[hw][1] += w01.y;
+                        acc[hw][2] += w23.x;
+                        acc[hw][3] += w23.y;
                     } else {
                         const uint16_t* vr0 =
                             reinterpret_cast<const uint16_t*>(st + size_t(srow0) * (C::ROW * 2) + C::RK * 2) + lane;
@@ -517,8 +515,7 @@ struct ProParams {
     const float* q;
     const int32_t* q_pos;
     const int32_t* seq_lens;
-    const float* w_up_k;
-    const float* mu_k;
+    const float* w_up_k_t;
     const float* rope_cos;
     const float* rope_sin;
     int32_t* P;
@@ -534,15 +531,7 @@ struct ProParams {
 
 template <class C>
 __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
-    // every block helps initialise the split records to "empty" (m = -inf, l = 0)
-    {
-        const size_t rec = size_t(p.RV) + 2;
-        const size_t nrec = p.n_record_floats / rec;
-        for (size_t r = size_t(blockIdx.x) * blockDim.x + threadIdx.x; r < nrec; r += size_t(gridDim.x) * blockDim.x) {
-            p.records[r * rec] = -INFINITY;
-            p.records[r * rec + 1] = 0.f;
-        }
-    }
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     if (blockIdx.x == 0) {
         // exclusive prefix of per-sequence tile counts (clamped lengths)
         __shared__ int32_t carry;
@@ -561,7 +550,6 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
             }
             const int tiles = (n + kTile - 1) / kTile;
             int v = tiles;  // inclusive warp scan
-            const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, v, o);
@@ -579,97 +567,101 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         if (threadIdx.x == 0) p.P[p.B] = carry;
         return;
     }
-    // (head, 16 sequences) block: this head's rows of the M_q images of those sequences
+    // one warp per (sequence, head): this head's rows of the sequence's M_q image
     constexpr int DH = C::DH, RK = C::RK, half = DH / 2, KC = DH / 8;
-    constexpr int ITEMS = ((RK + 1) * KC + 255) / 256;  // (row, 8-wide k chunk) items per thread
-    const int blk = blockIdx.x - 1;
-    const int h = blk % C::H, b0 = (blk / C::H) * kProSeqs;
-    extern __shared__ __align__(16) float wt[];  // [(RK + 1) * DH]: [n][i], W^K_up,t column n (n == RK: mu)
-    __shared__ __align__(16) float qr[DH];
-    __shared__ float red[8];
-    size_t w_off, mu_off;
-    if (p.variant == 0) {
-        w_off = ((size_t(p.layer) * C::H + h) * p.T + p.loop) * size_t(DH) * RK;
-        mu_off = (size_t(p.layer) * C::H + h) * size_t(p.T) * DH + size_t(p.loop) * DH;
-    } else {
-        w_off = ((size_t(p.layer) * p.T + p.loop) * C::H + h) * size_t(DH) * RK;
-        mu_off = size_t(p.layer) * p.T * C::H * DH + (size_t(p.loop) * C::H + h) * DH;
+    constexpr int NITEM = (RK + 1) * KC;  // (row, 8-wide k chunk) items
+    const int bh = (blockIdx.x - 1) * 8 + w;
+    if (bh >= p.B * C::H) return;
+    const int b = bh / C::H, h = bh - b * C::H;
+    __shared__ __align__(16) float qr_all[8][DH];
+    float* qr = qr_all[w];
+    const size_t slot = p.variant == 0 ? (size_t(p.layer) * C::H + h) * p.T + p.loop
+                                       : (size_t(p.layer) * p.T + p.loop) * C::H + h;
+    const float* wt = p.w_up_k_t + slot * size_t(RK + 1) * DH;  // [n][i], row RK = mu
+    int qp = p.q_pos[b];
+    if (qp < 0 || qp >= p.max_pos) {
+        qp = qp < 0 ? 0 : p.max_pos - 1;
+        if (h == 0 && lane == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
     }
-    for (int e = threadIdx.x; e < DH * RK; e += blockDim.x) {
-        const int i = e / RK, n = e % RK;
-        wt[n * DH + i] = p.w_up_k[w_off + e];
+    const float* qv = p.q + (size_t(b) * C::H + h) * DH;
+    for (int i = lane; i < half; i += 32) {
+        const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
+        const float lo = qv[i], hi = qv[i + half];
+        qr[i] = p.scale * (lo * c - hi * sn);
+        qr[i + half] = p.scale * (hi * c + lo * sn);
     }
-    for (int i = threadIdx.x; i < DH; i += blockDim.x) wt[RK * DH + i] = p.mu_k[mu_off + i];
+    __syncwarp();
+    // element (n, k): k < d/2: q'_k w_k + q'_{k+d/2} w_{k+d/2};  k >= d/2: q'_{i+d/2} w_i - q'_i w_{i+d/2}
+    auto item = [&](int e, float* v) {
+        const int n = e / KC, k0 = (e - n * KC) * 8;
+        const int i0 = k0 < half ? k0 : k0 - half;
+        const float4* wl = reinterpret_cast<const float4*>(wt + size_t(n) * DH + i0);
+        const float4* wh = reinterpret_cast<const float4*>(wt + size_t(n) * DH + i0 + half);
+        const float4* ql = reinterpret_cast<const float4*>(qr + i0);
+        const float4* qh = reinterpret_cast<const float4*>(qr + i0 + half);
+#pragma unroll
+        for (int u4 = 0; u4 < 2; ++u4) {
+            const float4 a = __ldg(wl + u4), bb = __ldg(wh + u4), x = ql[u4], y = qh[u4];
+            if (k0 < half) {
+                v[4 * u4 + 0] = x.x * a.x + y.x * bb.x;
+                v[4 * u4 + 1] = x.y * a.y + y.y * bb.y;
+                v[4 * u4 + 2] = x.z * a.z + y.z * bb.z;
+                v[4 * u4 + 3] = x.w * a.w + y.w * bb.w;
+            } else {
+                v[4 * u4 + 0] = y.x * a.x - x.x * bb.x;
+                v[4 * u4 + 1] = y.y * a.y - x.y * bb.y;
+                v[4 * u4 + 2] = y.z * a.z - x.z * bb.z;
+                v[4 * u4 + 3] = y.w * a.w - x.w * bb.w;
+            }
+        }
+    };
+    // small ranks: all of this lane's values stay in registers (one pass over W);
+    // large ranks: a max pass, then the values are recomputed for the write pass
+    constexpr int NPL = (NITEM + 31) / 32;  // items per lane
+    constexpr bool KEEP = NPL <= 12;
+    float keep[KEEP ? NPL : 1][8];
+    float mx = 0.f;
+#pragma unroll
+    for (int it = 0; it < NPL; ++it) {
+        const int e = lane + 32 * it;
+        if (e < NITEM) {
+            float* v = keep[KEEP ? it : 0];
+            item(e, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx = fmaxf(mx, fabsf(v[u]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
+    int e2 = 0;
+    float scale = 1.f;
+    if (mx > 0.f && isfinite(mx)) {
+        frexpf(mx, &e2);  // mx < 2^e2
+        scale = ldexpf(1.f, 15 - e2);
+    }
     const int part = h / C::HC, hc = h % C::HC, g = hc / C::HG, hg = hc % C::HG;
-    for (int b = b0; b < min(p.B, b0 + kProSeqs); ++b) {
-        int qp = p.q_pos[b];
-        if (qp < 0 || qp >= p.max_pos) {
-            qp = qp < 0 ? 0 : p.max_pos - 1;
-            if (h == 0 && threadIdx.x == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
-        }
-        __syncthreads();  // wt ready; previous sequence done with qr / red
-        const float* qv = p.q + (size_t(b) * C::H + h) * DH;
-        for (int i = threadIdx.x; i < half; i += blockDim.x) {
-            const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
-            const float lo = qv[i], hi = qv[i + half];
-            qr[i] = p.scale * (lo * c - hi * sn);
-            qr[i + half] = p.scale * (hi * c + lo * sn);
-        }
-        __syncthreads();
-        // element (n, k): k < d/2: q'_k w_k + q'_{k+d/2} w_{k+d/2};  k >= d/2: q'_{i+d/2} w_i - q'_i w_{i+d/2}
-        float val[ITEMS][8];
-        float mx = 0.f;
+    uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
 #pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int e = threadIdx.x + it * 256;
-            if (e < (RK + 1) * KC) {
-                const int n = e / KC, k0 = (e % KC) * 8;
-                const int i0 = k0 < half ? k0 : k0 - half;
-                const float* wn = wt + n * DH;
+    for (int it = 0; it < NPL; ++it) {
+        const int e = lane + 32 * it;
+        if (e >= NITEM) break;
+        float vv[8];
+        if (!KEEP) item(e, vv);
+        const float* v = KEEP ? keep[it] : vv;
+        const int n = e / KC, k0 = (e - n * KC) * 8;
+        const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
+        __align__(16) __half hv[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + u;
-                    const float wl = wn[i], wh = wn[i + half], ql = qr[i], qh = qr[i + half];
-                    val[it][u] = k0 < half ? ql * wl + qh * wh : qh * wl - ql * wh;
-                    mx = fmaxf(mx, fabsf(val[it][u]));
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-        __syncthreads();
-        mx = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red[i]);
-        // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
-        int e2 = 0;
-        float scale = 1.f;
-        if (mx > 0.f && isfinite(mx)) {
-            frexpf(mx, &e2);  // mx < 2^e2
-            scale = ldexpf(1.f, 15 - e2);
-        }
-        uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
-#pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int e = threadIdx.x + it * 256;
-            if (e < (RK + 1) * KC) {
-                const int n = e / KC, k0 = (e % KC) * 8;
-                const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
-                __align__(16) __half v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = __float2half_rn(val[it][u] * scale);
-                *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) =
-                    *reinterpret_cast<const uint4*>(v);
-            }
-        }
-        if (hg == 0)  // the group's padding rows
-            for (int e = threadIdx.x; e < (C::NG - C::HG * (RK + 1)) * KC; e += blockDim.x) {
-                const int rowi = C::HG * (RK + 1) + e / KC, k0 = (e % KC) * 8;
-                *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = make_uint4(0, 0, 0, 0);
-            }
-        if (threadIdx.x == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
+        for (int u = 0; u < 8; ++u) hv[u] = __float2half_rn(v[u] * scale);
+        *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = *reinterpret_cast<const uint4*>(hv);
     }
+    if (hg == 0)  // the group's padding rows
+        for (int e = lane; e < (C::NG - C::HG * (RK + 1)) * KC; e += 32) {
+            const int rowi = C::HG * (RK + 1) + e / KC, k0 = (e % KC) * 8;
+            *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = make_uint4(0, 0, 0, 0);
+        }
+    if (lane == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -733,8 +725,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.q = call.q;
     pp.q_pos = call.q_pos;
     pp.seq_lens = call.seq_lens;
-    pp.w_up_k = c->w_up_k;
-    pp.mu_k = c->mu_k;
+    pp.w_up_k_t = c->w_up_k_t;
     pp.rope_cos = c->rope_cos;
     pp.rope_sin = c->rope_sin;
     pp.P = reinterpret_cast<int32_t*>(ws + L.off_P);
@@ -761,9 +752,9 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.loop = call.loop;
     pp.variant = c->desc.variant;
     pp.scale = call.scale;
-    const int pro_smem = (C::RK + 1) * C::DH * int(sizeof(float));
-    LLA_CUDA_TRY(cudaFuncSetAttribute(tc_prologue_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, pro_smem));
-    tc_prologue_kernel<C><<<1 + C::H * ((B + kProSeqs - 1) / kProSeqs), 256, pro_smem, call.stream>>>(pp);
+    // split records start empty (l = 0); the combine skips them
+    LLA_CUDA_TRY(cudaMemsetAsync(pp.records, 0, pp.n_record_floats * sizeof(float), call.stream));
+    tc_prologue_kernel<C><<<1 + (B * C::H + 7) / 8, 256, 0, call.stream>>>(pp);
     LLA_CUDA_TRY(cudaGetLastError());
 
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).

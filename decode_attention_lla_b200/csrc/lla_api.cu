@@ -54,7 +54,7 @@ lla_status dev_alloc(T** p, size_t count) {
 void codec_free(lla_codec* c) {
     if (!c) return;
     void* ptrs[] = {c->w_up_k, c->w_up_v, c->mu_k, c->mu_v, c->bias_k, c->bias_v,
-                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles, c->status};
+                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles, c->status, c->w_up_k_t};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete c;
@@ -120,7 +120,7 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
         (st = dev_alloc(&c->bias_k, groups * rk)) || (st = dev_alloc(&c->bias_v, groups * rv)) ||
         (st = dev_alloc(&c->w_down_k_t, groups * rk * S)) || (st = dev_alloc(&c->w_down_v_t, groups * rv * S)) ||
         (st = dev_alloc(&c->rope_cos, nrope)) || (st = dev_alloc(&c->rope_sin, nrope)) ||
-        (st = dev_alloc(&c->status, 4))) {
+        (st = dev_alloc(&c->status, 4)) || (st = dev_alloc(&c->w_up_k_t, size_t(D) * T * H * (rk + 1) * d))) {
         codec_free(c);
         return st;
     }
@@ -155,7 +155,22 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
             rs[size_t(pos) * half + i] = float(sin(ang));
         }
     }
-    bool ok = cudaMemcpyAsync(c->w_up_k, w_up_k, nup_k * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+    // W^K_up,t transposed, mu^K_t appended as row r_k: [(layer, head, loop) slot][r_k + 1][d]
+    std::vector<float> wupt(size_t(D) * T * H * (rk + 1) * d);
+    for (int l = 0; l < D; ++l)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h) {
+                const size_t g = two_d ? (size_t(l) * T + t) * H + h : (size_t(l) * H + h) * T + t;
+                const float* W = w_up_k + g * size_t(d) * rk;
+                const float* m = two_d ? mu_k + size_t(l) * S + (size_t(t) * H + h) * d
+                                       : mu_k + (size_t(l) * H + h) * S + size_t(t) * d;
+                float* o = wupt.data() + g * size_t(rk + 1) * d;
+                for (int n = 0; n < rk; ++n)
+                    for (int i = 0; i < d; ++i) o[size_t(n) * d + i] = W[size_t(i) * rk + n];
+                for (int i = 0; i < d; ++i) o[size_t(rk) * d + i] = m[i];
+            }
+    bool ok = cudaMemcpyAsync(c->w_up_k_t, wupt.data(), wupt.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_up_k, w_up_k, nup_k * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->w_up_v, w_up_v, nup_v * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->mu_k, mu_k, nmu * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->mu_v, mu_v, nmu * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&

@@ -12,6 +12,9 @@ struct lla_codec {
     int device;
     // float32 copies
     float* w_up_k = nullptr;   // per-head [D][H][T][d][r_k];  2D [D][T][H][d][r_k]
+    // W^K_up,t transposed with mu^K_t appended as the last row, for the query prologue:
+    // per-head [D][H][T][r_k + 1][d];  2D [D][T][H][r_k + 1][d]
+    float* w_up_k_t = nullptr;
     float* w_up_v = nullptr;   // per-head [D][H][T][d][r_v];  2D [D][T][H][d][r_v]
     float* mu_k = nullptr;     // per-head [D][H][S];          2D [D][S]
     float* mu_v = nullptr;

@@ -196,6 +196,28 @@ __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) ----------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+// d = a * b + c, elementwise on the two lanes
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// both bf16 halves of a 32-bit word as an fp32 pair (low half first)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+    return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
 // layout: rows of 64 16-bit elements (128 B), 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
