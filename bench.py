@@ -60,6 +60,27 @@ def parse():
     return ap.parse_args()
 
 
+def rank_tag(workload: str, rank: int) -> str:
+    """Seed namespace of one rank: every rank decodes its own sequences (no shared data)."""
+    return f"bench/{workload}/rank{rank}"
+
+
+def max_over_ranks(ms: float, device) -> float:
+    """Max of a per-rank duration over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
+
+
 def rho_of(cfg):
     if cfg["variant"] == 0:
         return 2 * cfg["T"] * cfg["d_head"] / (cfg["r_k"] + cfg["r_v"])
@@ -234,7 +255,7 @@ def run_ours(a, cfg):
     T, D, H, d, rk, rv = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"]
     B, N = cfg["batch"], cfg["context"]
     cap = N + 1  # one free slot per sequence for the token appended by the step
-    tag = f"bench/{a.workload}/rank{rank}"
+    tag = rank_tag(a.workload, rank)
     codec_np = syn.seeded_codec(cfg, f"bench/{a.workload}/codec")
     desc = lla.Desc(D, T, H, d, rk, rv, cfg["variant"], cfg["rope_base"], cap + 1)
     codec = lla.Codec(desc, codec_np["w_down_k"], codec_np["w_down_v"], codec_np["w_up_k"], codec_np["w_up_v"],
@@ -313,12 +334,9 @@ def run_ours(a, cfg):
         dist.barrier()
     ms = g0.elapsed_time(g1)
     kern_ms = [e0.elapsed_time(e1) for row in ev_objs for e0, e1 in row]
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dev)
     ctx_tokens_step = B * N * T * D
-    value = world * ctx_tokens_step * a.steps / (ms_max / 1e3)
+    value = job_value(ctx_tokens_step, a.steps, world, ms_max)
 
     # end to end through the C ABI with host buffers: q in, out back, new-token stacks in
     e2e_value = None
@@ -339,10 +357,7 @@ def run_ours(a, cfg):
             step(host=host)
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e_value = world * ctx_tokens_step * a.e2e_steps / (float(e2e_ms.item()) / 1e3)
+        e2e_value = job_value(ctx_tokens_step, a.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), dev))
     h2d = T * D * B * H * d * 4 + int(np.prod(x_shape)) * 2
     d2h = T * D * B * H * d * 4
 
