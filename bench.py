@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling runs)")
+    ap.add_argument("--mode", choices=["decode", "encode"], default="decode",
+                    help="encode: time prefill encoding of teacher stacks instead of the decode step")
+    ap.add_argument("--encode-tokens", type=int, default=4096, help="tokens per encode call (encode mode)")
     return ap.parse_args()
 
 
@@ -396,7 +399,62 @@ def main():
         a.workload = f"{a.workload}[batch={cfg['batch']},layers={cfg['D']}]"
     if a.impl == "reference":
         return run_reference(a, cfg)
+    if a.mode == "encode":
+        return run_encode(a, cfg)
     return run_ours(a, cfg)
+
+
+def run_encode(a, cfg):
+    """Prefill throughput of lla_encode: stacks of n tokens for every layer -> latents.
+
+    One step encodes `--encode-tokens` tokens (all layers, heads and both axes) into
+    distinct store slots; the stacks are resident in HBM.  Reports tokens/s and the
+    HBM rate on the stacks, the bytes the encode must read.
+    """
+    import torch
+
+    import decode_attention_lla_b200 as lla
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    T, D, H, d, rk, rv = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"]
+    n = a.encode_tokens
+    codec_np = syn.seeded_codec(cfg, f"bench/{a.workload}/codec")
+    desc = lla.Desc(D, T, H, d, rk, rv, cfg["variant"], cfg["rope_base"], 16)
+    codec = lla.Codec(desc, codec_np["w_down_k"], codec_np["w_down_v"], codec_np["w_up_k"], codec_np["w_up_v"],
+                      codec_np["mu_k"], codec_np["mu_v"])
+    S = T * d if cfg["variant"] == 0 else T * H * d
+    x_shape = (n, D, H, 2, S) if cfg["variant"] == 0 else (n, D, 2, S)
+    x = torch.empty(x_shape, dtype=torch.bfloat16, device=dev)
+    x.normal_(generator=syn.torch_generator(f"bench/{a.workload}/enc_x", dev))
+    slots = 4
+    store = torch.empty(lla.store_bytes(desc, slots, n) // 2, dtype=torch.bfloat16, device=dev)
+    seq = torch.zeros(n, dtype=torch.int32, device=dev)
+    tok = torch.arange(n, dtype=torch.int32, device=dev)
+    for i in range(a.warmup):
+        seq.fill_(i % slots)
+        lla.encode(codec, x, n, 0, D, seq, tok, store, slots, n)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(a.steps):
+        seq.fill_(i % slots)
+        lla.encode(codec, x, n, 0, D, seq, tok, store, slots, n)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.steps
+    in_bytes = int(np.prod(x_shape)) * 2
+    peak, kind = measured_peak()
+    line = {"metric": "LLA encode: prefill tokens/s (all layers and heads)", "value": n / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(config_json(cfg, a.workload, 1), step=f"encode {n} tokens x {D} layers"),
+            "roofline": {"bound": "hbm", "achieved": in_bytes / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": in_bytes / (ms / 1e3) / 1e9 / peak, "traffic": None, "kernel": "lla encode",
+                         "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": in_bytes}}
+    print(json.dumps(line), flush=True)
+    codec.close()
+    return 0
 
 
 if __name__ == "__main__":

@@ -32,38 +32,62 @@ struct CombineParams {
     int tc_G, tc_parts, tc_hc;
 };
 
-// Record range [s0, s1) and record stride for (b, h).  In the tensor-core
-// layout, CTA c of G covers flattened tiles [c W / G, (c+1) W / G) with
-// W = parts * total; the CTA owning tile x is ((x + 1) G - 1) / W.
-__device__ __forceinline__ void record_range(const CombineParams& p, int b, int h, int& s0, int& s1, int& hrec,
-                                             int& hstride) {
-    if (p.tc_P) {
-        const int part = h / p.tc_hc;
-        hrec = h - part * p.tc_hc;
-        hstride = p.tc_hc;
+// The records of (b, h): rec(s) for s in [0, n).
+//   Split kernel: slots b*splits .. (b+1)*splits (or slot_range), record (slot * H + h).
+//   Tensor-core kernel: the CTAs form G/parts groups over the tile space; group g covers
+//   tiles [g total / groups, (g+1) total / groups), so the group owning tile x is
+//   ((x + 1) groups - 1) / total.  Group g's CTA for head part p writes record set
+//   id = (g + b) * parts + p, one record per TMEM lane quarter and head of the part:
+//   record ((id * 4 + quarter) * hc + head_in_part).
+struct RecordSet {
+    const float* base;
+    size_t rec_len;
+    int n;
+    // split kernel
+    int s0, hstride, hrec;
+    // tensor-core kernel
+    bool tc;
+    long long g0;
+    int b, part, parts, hc;
+    __device__ const float* rec(int s) const {
+        if (!tc) return base + (size_t(s0 + s) * hstride + hrec) * rec_len;
+        const long long id = (g0 + s / 4 + b) * parts + part;
+        return base + (size_t(id * 4 + (s & 3)) * hc + hrec) * rec_len;
+    }
+};
+
+__device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, int h) {
+    RecordSet r;
+    r.base = p.partials;
+    r.rec_len = lla_partial_floats(p.r_v);
+    r.tc = p.tc_P != nullptr;
+    r.b = b;
+    r.n = 0;
+    if (r.tc) {
+        r.parts = p.tc_parts;
+        r.hc = p.tc_hc;
+        r.part = h / p.tc_hc;
+        r.hrec = h - r.part * p.tc_hc;
         const long long total = p.tc_P[p.B];
         const int tiles = p.tc_P[b + 1] - p.tc_P[b];
-        if (tiles == 0 || total == 0) {
-            s0 = s1 = 0;
-            return;
-        }
-        const long long W = total * p.tc_parts;
-        const long long x0 = part * total + p.tc_P[b], x1 = x0 + tiles - 1;
-        const long long c0 = ((x0 + 1) * p.tc_G - 1) / W, c1 = ((x1 + 1) * p.tc_G - 1) / W;
-        const long long key = (long long)part * p.B + b;
-        s0 = int(4 * (key + c0));
-        s1 = int(4 * (key + c1 + 1));
-    } else if (p.slot_range) {
-        s0 = p.slot_range[2 * b];
-        s1 = p.slot_range[2 * b + 1];
-        hrec = h;
-        hstride = p.H;
+        const long long groups = p.tc_G / p.tc_parts;
+        if (tiles == 0 || total == 0 || groups == 0) return r;
+        const long long x0 = p.tc_P[b], x1 = x0 + tiles - 1;
+        r.g0 = ((x0 + 1) * groups - 1) / total;
+        const long long g1 = ((x1 + 1) * groups - 1) / total;
+        r.n = int(4 * (g1 - r.g0 + 1));
     } else {
-        s0 = b * p.splits;
-        s1 = s0 + p.splits;
-        hrec = h;
-        hstride = p.H;
+        r.hstride = p.H;
+        r.hrec = h;
+        if (p.slot_range) {
+            r.s0 = p.slot_range[2 * b];
+            r.n = p.slot_range[2 * b + 1] - r.s0;
+        } else {
+            r.s0 = b * p.splits;
+            r.n = p.splits;
+        }
     }
+    return r;
 }
 
 // One warp per (sequence, head); the CTA's sixteen warps share W^V_up,t of one head.
@@ -94,10 +118,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     __syncthreads();
     if (b >= p.B) return;
 
-    const size_t rec_len = lla_partial_floats(rv);
-    int s0, s1, hr, hs;
-    record_range(p, b, h, s0, s1, hr, hs);
-    auto rec = [&](int s) { return p.partials + (size_t(s) * hs + hr) * rec_len; };
+    const RecordSet rs = record_set(p, b, h);
+    auto rec = [&](int s) { return rs.rec(s); };
+    const int s0 = 0, s1 = rs.n;
     // merged maximum and normaliser over the records (log-sum-exp); a record with l = 0
     // saw no valid token and is skipped whatever its m holds
     float M = -INFINITY;

@@ -54,9 +54,12 @@ constexpr uint32_t kFlagTimeout = 4u;
 
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-template <int DH_, int RK_, int RV_, int H_>
+// TWO_D: LLA-2D codec, one latent row per token shared by all heads (otherwise one
+// row per (token, head)).
+template <int DH_, int RK_, int RV_, int H_, bool TWO_D_ = false>
 struct Cfg {
     static constexpr int DH = DH_, RK = RK_, RV = RV_, H = H_;
+    static constexpr bool TWO_D = TWO_D_;
     static constexpr int ROW = RK + RV;
     // heads per TMEM group: as many as fit N <= 256 (even, dividing H)
     static constexpr int HG = (16 * (RK + 1) <= 240 && H % 16 == 0) ? 16
@@ -70,19 +73,27 @@ struct Cfg {
     static constexpr int PARTS = H / HC;
     static constexpr int MQ_BYTES = GPC * MQ_GROUP_BYTES;
     static constexpr int PHI_BYTES = kTile * DH * 2;
+    // Phi tile buffers: two where the per-tile CUDA-core work is too short to hide a reload
+    static constexpr int NPHI = TWO_D ? 2 : 1;
     static constexpr int TOKS = (ROW * 2 * 128 <= 16384) ? 128 : (ROW * 2 * 64 <= 16384) ? 64 : 32;
     static constexpr int CHUNKS = kTile / TOKS;
     static constexpr int STAGE_BYTES = TOKS * ROW * 2;
     static constexpr int BAR_BYTES = 1024;
-    static constexpr int FIXED = 1024 /*align slack*/ + PHI_BYTES + MQ_BYTES + BAR_BYTES;
+    static constexpr int FIXED = 1024 /*align slack*/ + NPHI * PHI_BYTES + MQ_BYTES + BAR_BYTES;
     static constexpr int NST_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int NST = NST_RAW > 32 ? 32 : NST_RAW;
     static constexpr int SMEM = FIXED + NST * STAGE_BYTES;
     // compute warps: WPQ per TMEM lane quarter, each taking HG / WPQ heads of every group
-    static constexpr int WPQ = HG >= 4 ? 4 : HG;
+    static constexpr int WPQ = TWO_D ? (HC >= 4 ? 4 : HC) : (HG >= 4 ? 4 : HG);
     static constexpr int NCW = 4 * WPQ;
     static constexpr int THREADS = 32 * (2 + NCW);
     static constexpr int HPW = HC / WPQ;  // heads per compute warp
+    // latent stages per tile and the warps reading each stage: per-head rows give one stage
+    // per (head, token chunk), read by that head's warp of each quarter in the chunk; the 2D
+    // row is one stage per token chunk, read by every warp of those quarters
+    static constexpr int STAGES_PER_TILE = TWO_D ? CHUNKS : HC * CHUNKS;
+    static constexpr int ST_CONSUMERS = (TOKS / 32) * (TWO_D ? WPQ : 1);
+    static constexpr int H_MAP = TWO_D ? 1 : H;  // head extent of the latent tensor map
     static constexpr int TMEM_COLS = 512;
     // TMEM accumulator ring: as many NG-column buffers as fit in 512 columns (at most 4)
     static constexpr int NBUF = (512 / NG) > 4 ? 4 : (512 / NG);
@@ -95,7 +106,7 @@ struct Cfg {
     static constexpr int VPL = VQUAD ? 4 : RV / 32;           // accumulators per lane per head
     static_assert(DH % 64 == 0 && DH <= 256, "d_head must be a multiple of 64");
     static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
-    static_assert(H % HC == 0 && HG % WPQ == 0 && HG % 2 == 0, "head split");
+    static_assert(H % HC == 0 && HC % WPQ == 0 && HG % 2 == 0, "head split");
     static_assert(NG <= BUF_COLS, "TMEM buffer");
     static_assert(NST >= 2, "stages");
     static_assert(SMEM <= kSmemLimit, "shared memory");
@@ -113,45 +124,51 @@ struct TcParams {
     int B, G;
 };
 
-// Walks the CTA's contiguous share of the flattened (part, sequence, tile) space.
+// The CTAs form G / parts groups of `parts` CTAs; CTA c serves head part c % parts over the
+// tile range of group c / parts, a contiguous share of the flattened (sequence, tile) space.
+// The parts of a group walk the same tiles at the same time, so the LLA-2D latent row, read
+// by every part, comes from L2 after its first read.  A CTA writes one record set per
+// sequence it touches, with id (group + sequence) * parts + part: unique, since group and
+// sequence both rise along a walk.
 struct TileWalker {
     const int32_t* P;
-    int B;
+    int B, parts;
     long long x, x1, total;
-    int p, b, t;
-    __device__ void init(const int32_t* P_, int B_, int G, int cta, int parts) {
+    int p, gi, b, t;
+    __device__ void init(const int32_t* P_, int B_, int G, int cta, int parts_) {
         P = P_;
         B = B_;
+        parts = parts_;
         total = P[B];
-        const long long W = total * parts;
-        x = W * cta / G;
-        x1 = W * (cta + 1) / G;
+        const int groups = G / parts;
+        p = cta % parts;
+        gi = cta / parts;
+        x = x1 = 0;
+        if (gi >= groups) return;
+        x = total * gi / groups;
+        x1 = total * (gi + 1) / groups;
         if (x < x1) locate();
     }
     __device__ void locate() {
-        p = int(x / total);
-        const long long xt = x - p * total;
-        int lo = 0, hi = B - 1;  // largest b with P[b] <= xt
+        int lo = 0, hi = B - 1;  // largest b with P[b] <= x
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (P[mid] <= xt) lo = mid;
+            if (P[mid] <= x) lo = mid;
             else hi = mid - 1;
         }
         b = lo;
-        t = int(xt - P[b]);
+        t = int(x - P[b]);
     }
     __device__ bool valid() const { return x < x1; }
-    __device__ int key() const { return p * B + b; }
+    __device__ int key() const { return b; }  // M_q image and record set change with the sequence
+    __device__ long long record_id() const { return (long long)(gi + b) * parts + p; }
     __device__ void next() {
         ++x;
         if (x >= x1) return;
         ++t;
         while (t >= P[b + 1] - P[b]) {
             t = 0;
-            if (++b == B) {
-                b = 0;
-                ++p;
-            }
+            ++b;
         }
     }
 };
@@ -178,14 +195,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* phi_s = smem;
-    uint8_t* mq_s = phi_s + C::PHI_BYTES;
+    uint8_t* mq_s = phi_s + C::NPHI * C::PHI_BYTES;
     uint8_t* stage_s = mq_s + C::MQ_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage_s + C::NST * C::STAGE_BYTES);
-    uint64_t* phi_full = bars + 0;
-    uint64_t* phi_empty = bars + 1;
-    uint64_t* mq_full = bars + 2;
-    uint64_t* mq_empty = bars + 3;
-    uint64_t* tm_full = bars + 4;            // [NBUF]
+    uint64_t* phi_full = bars;                    // [NPHI]
+    uint64_t* phi_empty = bars + C::NPHI;         // [NPHI]
+    uint64_t* mq_full = bars + 2 * C::NPHI;
+    uint64_t* mq_empty = mq_full + 1;
+    uint64_t* tm_full = mq_full + 2;          // [NBUF]
     uint64_t* tm_empty = tm_full + C::NBUF;  // [NBUF]
     uint64_t* st_full = tm_empty + C::NBUF;  // [NST]
     uint64_t* st_empty = st_full + C::NST;
@@ -198,8 +215,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        mbar_init(phi_full, 1);
-        mbar_init(phi_empty, 1);
+        for (int i = 0; i < C::NPHI; ++i) {
+            mbar_init(phi_full + i, 1);
+            mbar_init(phi_empty + i, 1);
+        }
         mbar_init(mq_full, 1);
         mbar_init(mq_empty, 1);
         for (int i = 0; i < C::NBUF; ++i) {
@@ -208,7 +227,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         }
         for (int i = 0; i < C::NST; ++i) {
             mbar_init(st_full + i, 1);
-            mbar_init(st_empty + i, C::TOKS / 32);
+            mbar_init(st_empty + i, C::ST_CONSUMERS);
         }
         fence_mbar_init();
     }
@@ -238,7 +257,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 if (key != prev_key) {
                     if (mq_n > 0 && !(ok = mbar_wait(mq_empty, (mq_n - 1) & 1, p.status, kFlagTimeout, 1))) break;
                     mbar_expect_tx(mq_full, C::MQ_BYTES);
-                    const uint8_t* src = p.mq + size_t(key) * C::MQ_BYTES;
+                    const uint8_t* src = p.mq + (size_t(wk.p) * p.B + wk.b) * C::MQ_BYTES;
                     for (int off = 0; off < C::MQ_BYTES; off += 32768) {
                         const int n = C::MQ_BYTES - off < 32768 ? C::MQ_BYTES - off : 32768;
                         bulk_g2s(mq_s + off, src + off, n, mq_full, pol_keep);
@@ -246,12 +265,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     ++mq_n;
                     prev_key = key;
                 }
-                if (phi_n > 0 && !(ok = mbar_wait(phi_empty, (phi_n - 1) & 1, p.status, kFlagTimeout, 2))) break;
-                mbar_expect_tx(phi_full, C::PHI_BYTES);
-                bulk_g2s(phi_s, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES, phi_full, pol_keep);
-                ++phi_n;
-                for (int hl = 0; hl < C::HC && ok; ++hl) {
-                    const int h = wk.p * C::HC + hl;
+                {
+                    const uint32_t pb = phi_n % C::NPHI, pr = phi_n / C::NPHI;
+                    if (pr > 0 && !(ok = mbar_wait(phi_empty + pb, (pr - 1) & 1, p.status, kFlagTimeout, 2))) break;
+                    mbar_expect_tx(phi_full + pb, C::PHI_BYTES);
+                    bulk_g2s(phi_s + pb * C::PHI_BYTES, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES,
+                             phi_full + pb, pol_keep);
+                    ++phi_n;
+                }
+                for (int hl = 0; hl < (C::TWO_D ? 1 : C::HC) && ok; ++hl) {
+                    const int h = C::TWO_D ? 0 : wk.p * C::HC + hl;  // the 2D row has no head axis
                     for (int ch = 0; ch < C::CHUNKS; ++ch) {
                         const uint32_t slot = stage_k % C::NST, round = stage_k / C::NST;
                         if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
@@ -270,7 +293,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last issue into slot s
                 mbar_wait(st_full + s, (last / C::NST) & 1, p.status, kFlagTimeout, 4);
             }
-            if (phi_n > 0) mbar_wait(phi_full, (phi_n - 1) & 1, p.status, kFlagTimeout, 5);
+            for (uint32_t s = 0; s < C::NPHI && s < phi_n; ++s) {
+                const uint32_t last = phi_n - 1 - ((phi_n - 1 - s) % C::NPHI);  // last issue into buffer s
+                mbar_wait(phi_full + s, (last / C::NPHI) & 1, p.status, kFlagTimeout, 5);
+            }
             if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
         }
     } else if (warp == 1) {
@@ -291,8 +317,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     ++mq_n;
                     prev_key = key;
                 }
-                if (!(ok = mbar_wait(phi_full, phi_n & 1, p.status, kFlagTimeout, 8))) break;
+                const uint32_t pb = phi_n % C::NPHI;
+                if (!(ok = mbar_wait(phi_full + pb, (phi_n / C::NPHI) & 1, p.status, kFlagTimeout, 8))) break;
                 ++phi_n;
+                const uint32_t phi_buf = phi_addr + pb * C::PHI_BYTES;
                 tc_fence_after();
                 for (int g = 0; g < C::GPC && ok; ++g) {
                     const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
@@ -302,7 +330,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 #pragma unroll
                     for (int kk = 0; kk < C::DH / 16; ++kk) {
                         const uint32_t koff = uint32_t(kk & 3) * 32;  // 16-element K step inside the 64-wide swizzle atom
-                        const uint64_t ad = sw128_kmajor_desc(phi_addr + uint32_t(kk >> 2) * (kTile * 128) + koff);
+                        const uint64_t ad = sw128_kmajor_desc(phi_buf + uint32_t(kk >> 2) * (kTile * 128) + koff);
                         const uint64_t bd = sw128_kmajor_desc(mq_addr + g * C::MQ_GROUP_BYTES +
                                                               uint32_t(kk >> 2) * (C::NG * 128) + koff);
                         mma_f16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
@@ -310,7 +338,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     mma_commit(tm_full + buf);
                     ++gi;
                 }
-                mma_commit(phi_empty);
+                mma_commit(phi_empty + pb);
                 ++phi_commits;
             }
             if (prev_key != -1) {
@@ -318,7 +346,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 ++mq_commits;
             }
             // The commits' arrivals land in shared memory: see them complete before the CTA exits.
-            if (phi_commits > 0) mbar_wait(phi_empty, (phi_commits - 1) & 1, p.status, kFlagTimeout, 10);
+            for (uint32_t s = 0; s < C::NPHI && s < phi_commits; ++s) {
+                const uint32_t last = phi_commits - 1 - ((phi_commits - 1 - s) % C::NPHI);
+                mbar_wait(phi_empty + s, (last / C::NPHI) & 1, p.status, kFlagTimeout, 10);
+            }
             if (mq_commits > 0) mbar_wait(mq_empty, (mq_commits - 1) & 1, p.status, kFlagTimeout, 11);
         }
     } else {
@@ -330,19 +361,32 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         const uint32_t lane_addr = uint32_t(32 * qd) << 16;
         const int ch = (32 * qd) / C::TOKS;              // token chunk holding this quarter
         const int srow0 = 32 * qd - ch * C::TOKS;        // first stage row of this warp
-        constexpr int HH = C::HG / C::WPQ;               // heads per group handled by this warp
+        // this warp's heads: hl = hf + WPQ * i (i < HPW) of the CTA item's HC heads; head hl
+        // belongs to TMEM group hl / HG.  Heads of a group alternate between the warps of a
+        // quarter and each per-head stage is released right after use, so the stages in use
+        // stay adjacent in ring order and the rest of the ring keeps prefetching.
 
         float m[C::HPW], l[C::HPW], acc[C::HPW][C::VPL];
         const float* isc_row = p.inv_scale;  // per-(b, h) score scale, re-read from L1 when needed
         uint32_t gi = 0, tile_n = 0;
-        int prev_key = -1, prev_p = 0;
+        int prev_key = -1;
+        long long prev_id = 0;
         bool ok = true;
 
-        auto flush = [&](int key, int part) {
-            const long long id = (long long)blockIdx.x + key;
+        auto wait_stage = [&](uint32_t slot, uint32_t round) {
+            bool w_ok = true;
+            if (lane == 0) {
+                w_ok = ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14);
+                w_ok = w_ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13);
+            }
+            ok = __shfl_sync(0xffffffffu, w_ok, 0) && ok;
+            __syncwarp();  // lane 0's barrier acquire covers the whole warp's reads
+        };
+
+        auto flush = [&](long long id) {
 #pragma unroll
             for (int hw = 0; hw < C::HPW; ++hw) {
-                const int hl = (hw / HH) * C::HG + C::WPQ * (hw % HH) + hf;
+                const int hl = hf + C::WPQ * hw;
                 float* rec = p.records + ((size_t(id) * 4 + qd) * C::HC + hl) * size_t(C::RV + 2);
                 const float lsum = warp_sum(l[hw]);
                 float a[C::VPL];
@@ -364,72 +408,76 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     for (int v = 0; v < C::VPL; ++v) rec[2 + lane + 32 * v] = a[v];
                 }
             }
-            (void)part;
         };
 
         for (; wk.valid() && ok; wk.next(), ++tile_n) {
             const int key = wk.key();
             if (key != prev_key) {
-                if (prev_key != -1) flush(prev_key, prev_p);
+                if (prev_key != -1) flush(prev_id);
 #pragma unroll
                 for (int hw = 0; hw < C::HPW; ++hw) {
-                    const int hl = (hw / HH) * C::HG + C::WPQ * (hw % HH) + hf;
                     m[hw] = -INFINITY;
                     l[hw] = 0.f;
-                    (void)hl;
 #pragma unroll
                     for (int v = 0; v < C::VPL; ++v) acc[hw][v] = 0.f;
                 }
                 prev_key = key;
-                prev_p = wk.p;
+                prev_id = wk.record_id();
                 isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
             }
             const int valid = min(kTile, p.lens[wk.b] - wk.t * kTile);
             const bool row_ok = row < valid;
             const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this warp
 
-            for (int g = 0; g < C::GPC && ok; ++g) {
+            // the 2D stage (one latent row per token, shared by all heads) is held for the tile
+            uint32_t slot2d = 0;
+            if (C::TWO_D) {
+                const uint32_t sk = tile_n * C::STAGES_PER_TILE + ch;
+                slot2d = sk % C::NST;
+                wait_stage(slot2d, sk / C::NST);
+            }
+
+#pragma unroll
+            for (int g = 0; g < C::GPC; ++g) {
+                if (!ok) break;
                 const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
                 ok = __all_sync(0xffffffffu, mbar_wait(tm_full + buf, use & 1, p.status, kFlagTimeout, 12));
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
-                // Heads of the group alternate between the two warp halves (hg = 2 i + hf), one
-                // at a time, and each latent stage is released right after use: the stages in
-                // use are adjacent in ring order and the rest of the ring keeps prefetching.
 #pragma unroll
-                for (int i = 0; i < HH; ++i) {
-                    const int hg = C::WPQ * i + hf;         // head within the group
-                    const int hl = g * C::HG + hg;          // head within the CTA item
-                    const int hw = g * HH + i;              // this warp's head slot
-                    const uint32_t sk = tile_n * (C::HC * C::CHUNKS) + hl * C::CHUNKS + ch;
-                    const uint32_t slot = sk % C::NST, round = sk / C::NST;
-                    // score pieces from TMEM first: their latency overlaps the stage wait
-                    float gv[C::RK];
-                    float bias;
-                    tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
-#pragma unroll
-                    for (int a0 = 0; a0 < C::RK; a0 += 16) tmem_ld<16>(tcol + hg * C::RK + a0, &gv[a0]);
-                    bool w_ok = true;
-                    if (lane == 0) {
-                        w_ok = ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14);
-                        w_ok = w_ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13);
+                for (int hw = 0; hw < C::HPW; ++hw) {
+                    const int hl = hf + C::WPQ * hw;        // head within the CTA item
+                    if (hl / C::HG != g) continue;          // another group's head (warp-uniform)
+                    const int hg = hl - g * C::HG;          // head within the group
+                    uint32_t slot = slot2d;
+                    if (!C::TWO_D) {
+                        const uint32_t sk = tile_n * C::STAGES_PER_TILE + hl * C::CHUNKS + ch;
+                        slot = sk % C::NST;
+                        wait_stage(slot, sk / C::NST);
                     }
-                    ok = __shfl_sync(0xffffffffu, w_ok, 0) && ok;
-                    __syncwarp();  // lane 0's barrier acquire covers the whole warp's reads
-                    tmem_wait_ld();
                     const uint8_t* st = stage_s + size_t(slot) * C::STAGE_BYTES;
                     const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
 
-                    // ---- score: s = c^K . G + bias
-                    // packed fp32 pairs: two latent dimensions per f32x2 FMA, two independent chains
+                    // ---- score: s = c^K . G + bias, G read from TMEM 32 columns at a time;
+                    // packed fp32 pairs: two latent dimensions per f32x2 FMA, two chains
+                    float bias;
+                    tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
                     uint64_t s01 = 0, s23 = 0;
 #pragma unroll
-                    for (int a0 = 0; a0 < C::RK; a0 += 8) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(myrow + a0 * 2);
-                        s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[a0 + 0], gv[a0 + 1]), s01);
-                        s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[a0 + 2], gv[a0 + 3]), s23);
-                        s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[a0 + 4], gv[a0 + 5]), s01);
-                        s23 = f2_fma(bf16x2_to_f2(u.w), f2_pack(gv[a0 + 6], gv[a0 + 7]), s23);
+                    for (int a0 = 0; a0 < C::RK; a0 += 32) {
+                        constexpr int W = C::RK < 32 ? C::RK : 32;
+                        float gv[W];
+#pragma unroll
+                        for (int c0 = 0; c0 < W; c0 += 16) tmem_ld<16>(tcol + hg * C::RK + a0 + c0, &gv[c0]);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c0 = 0; c0 < W; c0 += 8) {
+                            const uint4 u = *reinterpret_cast<const uint4*>(myrow + (a0 + c0) * 2);
+                            s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[c0 + 0], gv[c0 + 1]), s01);
+                            s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[c0 + 2], gv[c0 + 3]), s23);
+                            s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[c0 + 4], gv[c0 + 5]), s01);
+                            s23 = f2_fma(bf16x2_to_f2(u.w), f2_pack(gv[c0 + 6], gv[c0 + 7]), s23);
+                        }
                     }
                     const float2 sp = f2_unpack(s01), sq = f2_unpack(s23);
                     const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * __ldg(isc_row + hl) : -INFINITY;
@@ -486,16 +534,22 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                             for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[32 * v]), acc[hw][v]);
                         }
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(st_empty + slot);
+                    if (!C::TWO_D) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(st_empty + slot);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tm_empty + buf);
                 ++gi;
             }
+            if (C::TWO_D) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(st_empty + slot2d);
+            }
         }
-        if (prev_key != -1) flush(prev_key, prev_p);
+        if (prev_key != -1) flush(prev_id);
     }
 
     tc_fence_before();
@@ -706,7 +760,9 @@ Layout tc_layout(int B, int G) {
 template <class C>
 int tc_grid(int override_ctas) {
     int g = override_ctas > 0 ? override_ctas : lla_num_sms();
-    return g > kMaxCtas ? kMaxCtas : g;
+    if (g > kMaxCtas) g = kMaxCtas;
+    if (g < C::PARTS) g = C::PARTS;  // at least one CTA per head part
+    return g - g % C::PARTS;         // whole groups of parts
 }
 
 template <class C>
@@ -758,10 +814,10 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     LLA_CUDA_TRY(cudaGetLastError());
 
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).
-    const size_t row_bytes = size_t(C::H) * C::ROW * 2;
+    const size_t row_bytes = size_t(C::H_MAP) * C::ROW * 2;  // one token of one layer
     CUtensorMap map;
     const void* base = call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
-    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(C::H), cuuint64_t(call.max_tokens), cuuint64_t(B)};
+    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(C::H_MAP), cuuint64_t(call.max_tokens), cuuint64_t(B)};
     cuuint64_t strides[3] = {cuuint64_t(C::ROW * 2), cuuint64_t(row_bytes),
                              cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
     cuuint32_t box[4] = {cuuint32_t(C::ROW), 1u, cuuint32_t(C::TOKS), 1u};
@@ -796,12 +852,14 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
 
 using CfgRho21 = Cfg<128, 16, 32, 16>;
 using CfgRho4 = Cfg<128, 96, 160, 16>;
+using Cfg2D = Cfg<128, 64, 128, 16, true>;
 
-enum class Which { none, rho21, rho4 };
+enum class Which { none, rho21, rho4, two_d };
 
 Which which(const lla_codec* c) {
     const lla_codec_desc& d = c->desc;
-    if (d.variant != 0 || d.d_head != 128 || d.H != 16) return Which::none;
+    if (d.d_head != 128 || d.H != 16) return Which::none;
+    if (d.variant == 1) return (d.r_k == 64 && d.r_v == 128) ? Which::two_d : Which::none;
     if (d.r_k == 16 && d.r_v == 32) return Which::rho21;
     if (d.r_k == 96 && d.r_v == 160) return Which::rho4;
     return Which::none;
@@ -815,6 +873,7 @@ size_t lla_tc_workspace_bytes(const lla_codec* c, int batch, int) {
     switch (which(c)) {
         case Which::rho21: return tc_layout<CfgRho21>(batch, kMaxCtas).total;
         case Which::rho4: return tc_layout<CfgRho4>(batch, kMaxCtas).total;
+        case Which::two_d: return tc_layout<Cfg2D>(batch, kMaxCtas).total;
         default: return 0;
     }
 }
@@ -823,6 +882,7 @@ lla_status lla_decode_tc(const lla_decode_call& call, int num_ctas) {
     switch (which(call.codec)) {
         case Which::rho21: return run_tc<CfgRho21>(call, num_ctas);
         case Which::rho4: return run_tc<CfgRho4>(call, num_ctas);
+        case Which::two_d: return run_tc<Cfg2D>(call, num_ctas);
         default: return LLA_ERR_UNSUPPORTED_SHAPE;
     }
 }

@@ -112,7 +112,6 @@ __global__ void __launch_bounds__(kThreads) encode_simt_kernel(EncodeParams p) {
 lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                              const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
                              int max_tokens, cudaStream_t stream) {
-    const lla_codec_desc& ds = c->desc;
     // the tensor-core kernel where it applies (TMA needs 16-byte aligned rows and stacks)
     if ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(store) & 15) == 0) {
         const lla_status st =

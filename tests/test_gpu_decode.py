@@ -142,11 +142,12 @@ def test_ragged_contexts_match_oracle(ci):
     lib.close()
 
 
+@pytest.mark.parametrize("ci", [1, 2])
 @pytest.mark.parametrize("impl,ctas", [(lla.IMPL_SIMT, 1), (lla.IMPL_SIMT, 2), (lla.IMPL_SIMT, 7),
                                        (lla.IMPL_TC, 1), (lla.IMPL_TC, 2), (lla.IMPL_TC, 7), (lla.IMPL_TC, 300)])
-def test_split_count_invariance(impl, ctas):
-    c = RAGGED[1]
-    cfg, codec, lib, bits, cK, cV, q = _ragged_case(c, "ragged1")
+def test_split_count_invariance(impl, ctas, ci):
+    c = RAGGED[ci]
+    cfg, codec, lib, bits, cK, cV, q = _ragged_case(c, f"ragged{ci}")
     if impl == lla.IMPL_TC and not _tc_supported(lib, c["B"], c["N"]):
         pytest.skip("tcgen05 kernel does not cover this shape")
     scale = 1 / math.sqrt(c["d_head"])
@@ -161,7 +162,9 @@ def test_split_count_invariance(impl, ctas):
 # ---------------------------------------------------------------------------------------------
 
 @pytest.mark.parametrize("c", [dict(D=2, T=2, H=4, d_head=16, r_k=12, r_v=20, B=3, N=200, lens=[200, 0, 77]),
-                               dict(D=1, T=4, H=16, d_head=128, r_k=64, r_v=128, B=2, N=300, lens=[300, 130])])
+                               dict(D=1, T=4, H=16, d_head=128, r_k=64, r_v=128, B=2, N=300, lens=[300, 130]),
+                               dict(D=2, T=4, H=16, d_head=128, r_k=64, r_v=128, B=5, N=900,
+                                    lens=[900, 0, 1, 385, 640])])
 def test_2d_matches_oracle(c):
     tag = f"2d/{c['d_head']}"
     cfg = dict(c, variant=1, rope_base=10000.0, mu_var=0.1)
@@ -174,11 +177,19 @@ def test_2d_matches_oracle(c):
                                    variant=1, rope_base=10000.0, max_pos=N + 4), codec)
     bits = to_bf16_bits(np.concatenate([cK, cV], -1))
     scale = 1 / math.sqrt(c["d_head"])
+    impls = [lla.IMPL_SIMT] + ([lla.IMPL_TC] if _tc_supported(lib, B, N) else [])
     for layer, loop in ((0, 0), (D - 1, c["T"] - 1)):
         ref = oracle_decode(codec, cfg, cK[:, layer], cV[:, layer], q, layer, loop, c["lens"], c["lens"], scale)
-        got, flags = _run(lib, bits, B, N, layer, loop, q, c["lens"], c["lens"], scale)
-        assert flags == 0
-        assert_close(got, ref, f"2d layer {layer} loop {loop}")
+        for impl in impls:
+            got, flags = _run(lib, bits, B, N, layer, loop, q, c["lens"], c["lens"], scale, impl=impl)
+            assert flags == 0
+            assert_close(got, ref, f"2d impl {impl} layer {layer} loop {loop}")
+            assert np.all(got[np.array(c["lens"]) == 0] == 0)
+        if lla.IMPL_TC in impls:  # result independent of the persistent grid
+            for ctas in (4, 8, 300):
+                got, _ = _run(lib, bits, B, N, layer, loop, q, c["lens"], c["lens"], scale, impl=lla.IMPL_TC,
+                              num_ctas=ctas)
+                assert_close(got, ref, f"2d tc ctas {ctas}")
     lib.close()
 
 

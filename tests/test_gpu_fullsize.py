@@ -63,3 +63,38 @@ def test_full_size_sampled(name, layer, loop, sample):
     del store, view
     lib.close()
     torch.cuda.empty_cache()
+
+
+def test_full_size_2d_sampled():
+    """LLA-2D at batch 256 x 8192 (19.3 GB store), one layer filled, sampled sequences."""
+    name, layer, loop, sample = "ouro_2d_b256_n8192", 11, 2, [0, 1, 128, 255]
+    cfg = syn.CONFIGS[name]
+    D, T, H, d, rk, rv = cfg["D"], cfg["T"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"]
+    B, N = cfg["batch"], cfg["context"]
+    cap = N + 1
+    codec = rounded_codec(syn.seeded_codec(cfg, f"full/{name}/codec"))
+    lib = lla.Codec(lla.Desc(D, T, H, d, rk, rv, 1, cfg["rope_base"], cap + 1), codec["w_down_k"],
+                    codec["w_down_v"], codec["w_up_k"], codec["w_up_v"], codec["mu_k"], codec["mu_v"])
+    store = torch.empty(lla.store_bytes(lib.desc, B, cap) // 2, dtype=torch.bfloat16, device=DEV)
+    view = store.view(B, D, cap, rk + rv)
+    view[:, layer].normal_(generator=syn.torch_generator(f"full/{name}/lat", DEV))
+    q = torch.empty(B, H, d, device=DEV).normal_(generator=syn.torch_generator(f"full/{name}/q", DEV))
+    lens_np = np.full(B, N, np.int32)
+    lens_np[sample[-1]] = N - 1000
+    lens = torch.from_numpy(lens_np).to(DEV)
+    out = torch.empty(B, H, d, device=DEV)
+    ws = torch.empty(lib.workspace_bytes(B, cap), dtype=torch.uint8, device=DEV)
+    scale = 1 / math.sqrt(d)
+    lla.decode_attn_2d(lib, store, B, cap, layer, loop, q, lens, lens, scale, out, ws)
+    torch.cuda.synchronize()
+    assert lla.workspace_flags(ws) == 0
+    got = out.cpu().numpy().astype(np.float64)
+    idx = torch.tensor(sample, device=DEV)
+    lat = view[idx, layer].float().cpu().numpy().astype(np.float64)  # [S, cap, rk+rv]
+    qs = q[idx].cpu().numpy().astype(np.float64)
+    ref = oracle_decode(codec, cfg, lat[..., :rk], lat[..., rk:], qs, layer, loop, lens_np[sample],
+                        lens_np[sample], scale)
+    assert_close(got[sample], ref, name)
+    del store, view
+    lib.close()
+    torch.cuda.empty_cache()
