@@ -31,6 +31,7 @@
 //               record per (segment, quarter, head) for the combine kernel.
 // Every wait is bounded (see sm100.cuh); a timeout sets a status bit.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
 #include <string.h>
@@ -54,13 +55,12 @@ constexpr uint32_t kFlagTimeout = 4u;
 
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// TWO_D: LLA-2D codec, one latent row per token shared by all heads (otherwise one
-// row per (token, head)).
-template <int DH_, int RK_, int RV_, int H_, bool TWO_D_ = false>
-struct Cfg {
+// Head grouping shared by both kernels: which heads share one score GEMM (a TMEM group,
+// N <= 256 columns), how many groups stay resident per CTA (their M_q images), and so how
+// many CTAs ("parts") split the heads of a tile.
+template <int DH_, int RK_, int RV_, int H_>
+struct HeadGroups {
     static constexpr int DH = DH_, RK = RK_, RV = RV_, H = H_;
-    static constexpr bool TWO_D = TWO_D_;
-    static constexpr int ROW = RK + RV;
     // heads per TMEM group: as many as fit N <= 256 (even, dividing H)
     static constexpr int HG = (16 * (RK + 1) <= 240 && H % 16 == 0) ? 16
                               : (8 * (RK + 1) <= 240 && H % 8 == 0) ? 8
@@ -73,40 +73,45 @@ struct Cfg {
     static constexpr int PARTS = H / HC;
     static constexpr int MQ_BYTES = GPC * MQ_GROUP_BYTES;
     static constexpr int PHI_BYTES = kTile * DH * 2;
-    // Phi tile buffers: two where the per-tile CUDA-core work is too short to hide a reload
-    static constexpr int NPHI = TWO_D ? 2 : 1;
+    static constexpr uint32_t IDESC = idesc_f16_f32(128, NG);
+    static_assert(DH % 64 == 0 && DH <= 256, "d_head must be a multiple of 64");
+    static_assert(H % HC == 0 && HG % 2 == 0, "head split");
+};
+
+// Per-head latent rows (one row of r_k + r_v per (token, head)).
+template <int DH_, int RK_, int RV_, int H_>
+struct Cfg : HeadGroups<DH_, RK_, RV_, H_> {
+    using HG_ = HeadGroups<DH_, RK_, RV_, H_>;
+    using HG_::DH, HG_::RK, HG_::RV, HG_::H, HG_::HG, HG_::NG, HG_::HC, HG_::MQ_BYTES, HG_::PHI_BYTES;
+    static constexpr bool TWO_D = false;
+    static constexpr int ROW = RK + RV;
     static constexpr int TOKS = (ROW * 2 * 128 <= 16384) ? 128 : (ROW * 2 * 64 <= 16384) ? 64 : 32;
     static constexpr int CHUNKS = kTile / TOKS;
     static constexpr int STAGE_BYTES = TOKS * ROW * 2;
     static constexpr int BAR_BYTES = 1024;
-    static constexpr int FIXED = 1024 /*align slack*/ + NPHI * PHI_BYTES + MQ_BYTES + BAR_BYTES;
+    static constexpr int FIXED = 1024 /*align slack*/ + PHI_BYTES + MQ_BYTES + BAR_BYTES;
     static constexpr int NST_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int NST = NST_RAW > 32 ? 32 : NST_RAW;
     static constexpr int SMEM = FIXED + NST * STAGE_BYTES;
     // compute warps: WPQ per TMEM lane quarter, each taking HG / WPQ heads of every group
-    static constexpr int WPQ = TWO_D ? (HC >= 4 ? 4 : HC) : (HG >= 4 ? 4 : HG);
+    static constexpr int WPQ = HG >= 4 ? 4 : HG;
     static constexpr int NCW = 4 * WPQ;
     static constexpr int THREADS = 32 * (2 + NCW);
     static constexpr int HPW = HC / WPQ;  // heads per compute warp
-    // latent stages per tile and the warps reading each stage: per-head rows give one stage
-    // per (head, token chunk), read by that head's warp of each quarter in the chunk; the 2D
-    // row is one stage per token chunk, read by every warp of those quarters
-    static constexpr int STAGES_PER_TILE = TWO_D ? CHUNKS : HC * CHUNKS;
-    static constexpr int ST_CONSUMERS = (TOKS / 32) * (TWO_D ? WPQ : 1);
-    static constexpr int H_MAP = TWO_D ? 1 : H;  // head extent of the latent tensor map
+    // one stage per (head, token chunk), read by that head's warp of each quarter in the chunk
+    static constexpr int STAGES_PER_TILE = HC * CHUNKS;
+    static constexpr int ST_CONSUMERS = TOKS / 32;
     static constexpr int TMEM_COLS = 512;
     // TMEM accumulator ring: as many NG-column buffers as fit in 512 columns (at most 4)
     static constexpr int NBUF = (512 / NG) > 4 ? 4 : (512 / NG);
     static constexpr int BUF_COLS = (512 / NBUF) / 16 * 16;
-    static constexpr uint32_t IDESC = idesc_f16_f32(128, NG);
     // V-side lane mapping
     static constexpr bool VQUAD = (RV == 32 || RV == 64 || RV == 128);
     static constexpr int VAL = VQUAD ? RV / 4 : 32;          // lanes along the latent dimension
     static constexpr int VTL = 32 / VAL;                      // token sub-lanes
     static constexpr int VPL = VQUAD ? 4 : RV / 32;           // accumulators per lane per head
-    static_assert(DH % 64 == 0 && DH <= 256, "d_head must be a multiple of 64");
     static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
-    static_assert(H % HC == 0 && HC % WPQ == 0 && HG % 2 == 0, "head split");
+    static_assert(HC % WPQ == 0, "head split");
     static_assert(NG <= BUF_COLS, "TMEM buffer");
     static_assert(NST >= 2, "stages");
     static_assert(SMEM <= kSmemLimit, "shared memory");
@@ -195,12 +200,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* phi_s = smem;
-    uint8_t* mq_s = phi_s + C::NPHI * C::PHI_BYTES;
+    uint8_t* mq_s = phi_s + C::PHI_BYTES;
     uint8_t* stage_s = mq_s + C::MQ_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage_s + C::NST * C::STAGE_BYTES);
-    uint64_t* phi_full = bars;                    // [NPHI]
-    uint64_t* phi_empty = bars + C::NPHI;         // [NPHI]
-    uint64_t* mq_full = bars + 2 * C::NPHI;
+    uint64_t* phi_full = bars;
+    uint64_t* phi_empty = bars + 1;
+    uint64_t* mq_full = bars + 2;
     uint64_t* mq_empty = mq_full + 1;
     uint64_t* tm_full = mq_full + 2;          // [NBUF]
     uint64_t* tm_empty = tm_full + C::NBUF;  // [NBUF]
@@ -215,10 +220,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::NPHI; ++i) {
-            mbar_init(phi_full + i, 1);
-            mbar_init(phi_empty + i, 1);
-        }
+        mbar_init(phi_full, 1);
+        mbar_init(phi_empty, 1);
         mbar_init(mq_full, 1);
         mbar_init(mq_empty, 1);
         for (int i = 0; i < C::NBUF; ++i) {
@@ -265,16 +268,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     ++mq_n;
                     prev_key = key;
                 }
-                {
-                    const uint32_t pb = phi_n % C::NPHI, pr = phi_n / C::NPHI;
-                    if (pr > 0 && !(ok = mbar_wait(phi_empty + pb, (pr - 1) & 1, p.status, kFlagTimeout, 2))) break;
-                    mbar_expect_tx(phi_full + pb, C::PHI_BYTES);
-                    bulk_g2s(phi_s + pb * C::PHI_BYTES, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES,
-                             phi_full + pb, pol_keep);
-                    ++phi_n;
-                }
-                for (int hl = 0; hl < (C::TWO_D ? 1 : C::HC) && ok; ++hl) {
-                    const int h = C::TWO_D ? 0 : wk.p * C::HC + hl;  // the 2D row has no head axis
+                if (phi_n > 0 && !(ok = mbar_wait(phi_empty, (phi_n - 1) & 1, p.status, kFlagTimeout, 2))) break;
+                mbar_expect_tx(phi_full, C::PHI_BYTES);
+                bulk_g2s(phi_s, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES, phi_full, pol_keep);
+                ++phi_n;
+                for (int hl = 0; hl < C::HC && ok; ++hl) {
+                    const int h = wk.p * C::HC + hl;
                     for (int ch = 0; ch < C::CHUNKS; ++ch) {
                         const uint32_t slot = stage_k % C::NST, round = stage_k / C::NST;
                         if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
@@ -293,10 +292,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last issue into slot s
                 mbar_wait(st_full + s, (last / C::NST) & 1, p.status, kFlagTimeout, 4);
             }
-            for (uint32_t s = 0; s < C::NPHI && s < phi_n; ++s) {
-                const uint32_t last = phi_n - 1 - ((phi_n - 1 - s) % C::NPHI);  // last issue into buffer s
-                mbar_wait(phi_full + s, (last / C::NPHI) & 1, p.status, kFlagTimeout, 5);
-            }
+            if (phi_n > 0) mbar_wait(phi_full, (phi_n - 1) & 1, p.status, kFlagTimeout, 5);
             if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
         }
     } else if (warp == 1) {
@@ -317,10 +313,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     ++mq_n;
                     prev_key = key;
                 }
-                const uint32_t pb = phi_n % C::NPHI;
-                if (!(ok = mbar_wait(phi_full + pb, (phi_n / C::NPHI) & 1, p.status, kFlagTimeout, 8))) break;
+                if (!(ok = mbar_wait(phi_full, phi_n & 1, p.status, kFlagTimeout, 8))) break;
                 ++phi_n;
-                const uint32_t phi_buf = phi_addr + pb * C::PHI_BYTES;
                 tc_fence_after();
                 for (int g = 0; g < C::GPC && ok; ++g) {
                     const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
@@ -330,7 +324,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 #pragma unroll
                     for (int kk = 0; kk < C::DH / 16; ++kk) {
                         const uint32_t koff = uint32_t(kk & 3) * 32;  // 16-element K step inside the 64-wide swizzle atom
-                        const uint64_t ad = sw128_kmajor_desc(phi_buf + uint32_t(kk >> 2) * (kTile * 128) + koff);
+                        const uint64_t ad = sw128_kmajor_desc(phi_addr + uint32_t(kk >> 2) * (kTile * 128) + koff);
                         const uint64_t bd = sw128_kmajor_desc(mq_addr + g * C::MQ_GROUP_BYTES +
                                                               uint32_t(kk >> 2) * (C::NG * 128) + koff);
                         mma_f16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
@@ -338,7 +332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     mma_commit(tm_full + buf);
                     ++gi;
                 }
-                mma_commit(phi_empty + pb);
+                mma_commit(phi_empty);
                 ++phi_commits;
             }
             if (prev_key != -1) {
@@ -346,10 +340,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 ++mq_commits;
             }
             // The commits' arrivals land in shared memory: see them complete before the CTA exits.
-            for (uint32_t s = 0; s < C::NPHI && s < phi_commits; ++s) {
-                const uint32_t last = phi_commits - 1 - ((phi_commits - 1 - s) % C::NPHI);
-                mbar_wait(phi_empty + s, (last / C::NPHI) & 1, p.status, kFlagTimeout, 10);
-            }
+            if (phi_commits > 0) mbar_wait(phi_empty, (phi_commits - 1) & 1, p.status, kFlagTimeout, 10);
             if (mq_commits > 0) mbar_wait(mq_empty, (mq_commits - 1) & 1, p.status, kFlagTimeout, 11);
         }
     } else {
@@ -429,14 +420,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
             const bool row_ok = row < valid;
             const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this warp
 
-            // the 2D stage (one latent row per token, shared by all heads) is held for the tile
-            uint32_t slot2d = 0;
-            if (C::TWO_D) {
-                const uint32_t sk = tile_n * C::STAGES_PER_TILE + ch;
-                slot2d = sk % C::NST;
-                wait_stage(slot2d, sk / C::NST);
-            }
-
 #pragma unroll
             for (int g = 0; g < C::GPC; ++g) {
                 if (!ok) break;
@@ -449,12 +432,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     const int hl = hf + C::WPQ * hw;        // head within the CTA item
                     if (hl / C::HG != g) continue;          // another group's head (warp-uniform)
                     const int hg = hl - g * C::HG;          // head within the group
-                    uint32_t slot = slot2d;
-                    if (!C::TWO_D) {
-                        const uint32_t sk = tile_n * C::STAGES_PER_TILE + hl * C::CHUNKS + ch;
-                        slot = sk % C::NST;
-                        wait_stage(slot, sk / C::NST);
-                    }
+                    const uint32_t sk = tile_n * C::STAGES_PER_TILE + hl * C::CHUNKS + ch;
+                    const uint32_t slot = sk % C::NST;
+                    wait_stage(slot, sk / C::NST);
                     const uint8_t* st = stage_s + size_t(slot) * C::STAGE_BYTES;
                     const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
 
@@ -534,19 +514,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                             for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[32 * v]), acc[hw][v]);
                         }
                     }
-                    if (!C::TWO_D) {
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(st_empty + slot);
-                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(st_empty + slot);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tm_empty + buf);
                 ++gi;
-            }
-            if (C::TWO_D) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(st_empty + slot2d);
             }
         }
         if (prev_key != -1) flush(prev_id);
@@ -560,6 +534,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
+
+#include "decode_tc2d.cuh"
 
 // ---------------------------------------------------------------------------------------------
 // Prologue: tile plan, per-(sequence, head) M_q images, record initialisation.
@@ -813,17 +789,32 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tc_prologue_kernel<C><<<1 + (B * C::H + 7) / 8, 256, 0, call.stream>>>(pp);
     LLA_CUDA_TRY(cudaGetLastError());
 
-    // Tensor map over the layer's latents: dims (row elems, head, token, sequence).
-    const size_t row_bytes = size_t(C::H_MAP) * C::ROW * 2;  // one token of one layer
+    // Tensor map over the layer's latents: dims (row elems, head, token, sequence).  Per-head
+    // rows load whole (r_k + r_v) rows of TOKS tokens; the 2D row loads 64-element panels of
+    // 32 tokens in the 128-byte swizzle that the tensor-core operands use.
+    const int h_map = C::TWO_D ? 1 : C::H;
+    const size_t row_bytes = size_t(h_map) * C::ROW * 2;  // one token of one layer
     CUtensorMap map;
     const void* base = call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
-    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(C::H_MAP), cuuint64_t(call.max_tokens), cuuint64_t(B)};
+    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(h_map), cuuint64_t(call.max_tokens), cuuint64_t(B)};
     cuuint64_t strides[3] = {cuuint64_t(C::ROW * 2), cuuint64_t(row_bytes),
                              cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
-    cuuint32_t box[4] = {cuuint32_t(C::ROW), 1u, cuuint32_t(C::TOKS), 1u};
+    cuuint32_t box[4];
+    CUtensorMapSwizzle swz;
+    if constexpr (C::TWO_D) {
+        box[0] = 64u;
+        box[2] = cuuint32_t(C::QTOK);
+        swz = CU_TENSOR_MAP_SWIZZLE_128B;
+    } else {
+        box[0] = cuuint32_t(C::ROW);
+        box[2] = cuuint32_t(C::TOKS);
+        swz = CU_TENSOR_MAP_SWIZZLE_NONE;
+    }
+    box[1] = 1u;
+    box[3] = 1u;
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return LLA_ERR_CUDA;
 
@@ -837,9 +828,12 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tp.status = pp.status;
     tp.B = B;
     tp.G = G;
-    LLA_CUDA_TRY(cudaFuncSetAttribute(tc_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    void (*kernel)(const CUtensorMap, TcParams);
+    if constexpr (C::TWO_D) kernel = tc2d_decode_kernel<C>;
+    else kernel = tc_decode_kernel<C>;
+    LLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     if (call.ev_begin) LLA_CUDA_TRY(cudaEventRecord(call.ev_begin, call.stream));
-    tc_decode_kernel<C><<<G, C::THREADS, C::SMEM, call.stream>>>(map, tp);
+    kernel<<<G, C::THREADS, C::SMEM, call.stream>>>(map, tp);
     LLA_CUDA_TRY(cudaGetLastError());
     if (call.ev_end) LLA_CUDA_TRY(cudaEventRecord(call.ev_end, call.stream));
     lla_tc_ranges ranges;
@@ -852,7 +846,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
 
 using CfgRho21 = Cfg<128, 16, 32, 16>;
 using CfgRho4 = Cfg<128, 96, 160, 16>;
-using Cfg2D = Cfg<128, 64, 128, 16, true>;
+using Cfg2D = Cfg2<128, 64, 128, 16>;
 
 enum class Which { none, rho21, rho4, two_d };
 

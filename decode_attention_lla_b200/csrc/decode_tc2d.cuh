@@ -1,0 +1,482 @@
+// LLA-2D tensor-core decode kernel for sm_100a (part of the decode_tc.cu translation unit).
+//
+// [LLA §3, "LLA-2D"]: one latent row (c^K_j | c^V_j) per (sequence, layer, token) serves
+// all H heads; the per-(loop, head) up-projections differ.  Scores use the same bilinear
+// form as the per-head kernel, G = Phi M_q per group of heads on tcgen05 and an r_k-long
+// CUDA-core dot c^K_j . G_j per (token, head).  Because c^V_j is shared by the heads, the
+// latent-space V accumulation of [LLA §3 eq. (3)],
+//   acc_h += sum_j p_{h,j} c^V_j,
+// is itself a GEMM here: per 128-token tile,
+//   D [r_v x 16] = (C^V)^T [r_v x 128 tokens] . P [128 tokens x 16]
+// with C^V the MN-major operand straight from the TMA stage and P the bf16 probabilities.
+// Each 32-token quarter of a tile keeps its own online-softmax state (as in the per-head
+// kernel), so the 16 columns are (head of the CTA item, token quarter) and P is block
+// diagonal: quarter q's tokens feed only its own columns, and the other entries stay zero.
+// The compute warps then rescale and add D into registers: acc_{q,h} = alpha acc_{q,h} + D.
+//
+// Warp roles (one CTA per SM, persistent over the (head part, sequence, tile) walk):
+//   warp 0      TMA: M_q images (per sequence and part), Phi tiles (two buffers), c^K
+//               quarter slots (one 128-byte swizzled row per token).
+//   warp 1      TMEM allocator and MMA issuer: per tile the score GEMMs of every head
+//               group, then the V GEMM of the previous tile (its P is complete by then).
+//   warp 2      TMA: c^V quarter slots (two 64-wide swizzled panels per token).
+//   warps 3-18  compute: one warp per (TMEM lane quarter, head of the item).  Per tile:
+//               score, softmax, P and alpha into shared memory, then the previous tile's
+//               V GEMM result into its accumulators.
+// Every wait is bounded and sets a status bit on timeout.
+
+template <int DH_, int RK_, int RV_, int H_>
+struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
+    using HB = HeadGroups<DH_, RK_, RV_, H_>;
+    using HB::DH, HB::RK, HB::RV, HB::H, HB::HG, HB::NG, HB::HC, HB::GPC, HB::MQ_BYTES, HB::MQ_GROUP_BYTES,
+        HB::PHI_BYTES;
+    static constexpr bool TWO_D = true;
+    static constexpr int ROW = RK + RV;
+    static constexpr int QTOK = 32;                     // tokens per TMEM lane quarter
+    static constexpr int PANEL = QTOK * 128;            // one 64-wide swizzled panel of a quarter
+    static constexpr int K_SLOT = PANEL;                // c^K of a quarter (r_k = 64)
+    static constexpr int V_PANELS = RV / 64;
+    static constexpr int V_SLOT = V_PANELS * PANEL;     // c^V of a quarter
+    static constexpr int NPHI = 2;
+    static constexpr int VN = 16;                       // V GEMM columns: (head, quarter)
+    static constexpr int P_BYTES = (kTile / 64) * VN * 128;  // [token panel][16 rows][128 B]
+    static constexpr int BAR_BYTES = 1024;
+    static constexpr int FIXED = 1024 /*align slack*/ + NPHI * PHI_BYTES + MQ_BYTES + 2 * P_BYTES + BAR_BYTES;
+    static constexpr int NK = 8;                        // c^K ring: two tiles
+    static constexpr int NV_RAW = (kSmemLimit - FIXED - NK * K_SLOT) / V_SLOT;
+    static constexpr int NV = NV_RAW > 16 ? 16 : NV_RAW;
+    static constexpr int SMEM = FIXED + NK * K_SLOT + NV * V_SLOT;
+    static constexpr int NCW = 4 * HC;                  // one compute warp per (quarter, head)
+    static constexpr int THREADS = 32 * (3 + NCW);
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int NBUF = 3;                      // score accumulator ring
+    static constexpr int BUF_COLS = NG;
+    static constexpr int VCOL = NBUF * BUF_COLS;        // two V accumulators after the ring
+    static constexpr uint32_t IDESC_V = idesc_bf16_f32(128, VN, /*A MN-major*/ true, false);
+    static_assert(RK == 64, "c^K quarter slot is one 128-byte row per token");
+    static_assert(RV == 128, "the V GEMM has M = r_v = 128");
+    static_assert(HC * 4 == VN, "V GEMM columns = heads of the item x quarters");
+    static_assert(VCOL + 2 * VN <= TMEM_COLS, "TMEM columns");
+    static_assert(NV >= 4, "c^V ring");
+    static_assert(SMEM <= kSmemLimit, "shared memory");
+    static_assert((6 + 2 * NBUF + 6 + 2 * NK + 2 * NV) * 8 + 256 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
+    static_assert(1 + NK + NV <= 64, "issue counters");
+};
+
+// Wait for the last phase of each of `ns` ring barriers after `count` uses in ring order.
+__device__ __forceinline__ void wait_last_phases(uint64_t* bars, uint32_t ns, uint32_t count, uint32_t* status,
+                                                 uint32_t site) {
+    for (uint32_t s = 0; s < ns && s < count; ++s) {
+        const uint32_t last = count - 1 - ((count - 1 - s) % ns);
+        mbar_wait(bars + s, (last / ns) & 1, status, kFlagTimeout, site);
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
+                                                                  TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* phi_s = smem;                               // [NPHI][PHI_BYTES]
+    uint8_t* mq_s = phi_s + C::NPHI * C::PHI_BYTES;      // [GPC][MQ_GROUP_BYTES]
+    uint8_t* p_s = mq_s + C::MQ_BYTES;                   // [2][P_BYTES]
+    uint8_t* k_s = p_s + 2 * C::P_BYTES;                 // [NK][K_SLOT]
+    uint8_t* v_s = k_s + C::NK * C::K_SLOT;              // [NV][V_SLOT]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(v_s + C::NV * C::V_SLOT);
+    uint64_t* phi_full = bars;                // [2]
+    uint64_t* phi_empty = bars + 2;           // [2]
+    uint64_t* mq_full = bars + 4;
+    uint64_t* mq_empty = bars + 5;
+    uint64_t* tm_full = bars + 6;             // [NBUF]
+    uint64_t* tm_empty = tm_full + C::NBUF;   // [NBUF]
+    uint64_t* p_full = tm_empty + C::NBUF;    // [2] P and alpha of a tile written
+    uint64_t* d_full = p_full + 2;            // [2] V GEMM of a tile complete
+    uint64_t* d_empty = d_full + 2;           // [2] V accumulator read by every compute warp
+    uint64_t* k_full = d_empty + 2;           // [NK]
+    uint64_t* k_empty = k_full + C::NK;
+    uint64_t* v_full = k_empty + C::NK;       // [NV]
+    uint64_t* v_empty = v_full + C::NV;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_empty + C::NV);
+    // loads issued per slot (a consumer first waits for its round to be issued, so that a
+    // parity wait cannot match an earlier round of the slot)
+    volatile uint32_t* k_issued = tmem_holder + 1;
+    volatile uint32_t* v_issued = k_issued + C::NK;
+    float* alpha_s = reinterpret_cast<float*>(tmem_holder + 64);  // [2][4 quarters][HC]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < C::NK) k_issued[threadIdx.x] = 0;
+    if (threadIdx.x < C::NV) v_issued[threadIdx.x] = 0;
+    // P starts all zero: each compute warp only ever writes its own block of it
+    for (int i = threadIdx.x; i < 2 * C::P_BYTES / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(p_s)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(phi_full + i, 1);
+            mbar_init(phi_empty + i, 1);
+            mbar_init(p_full + i, C::NCW);
+            mbar_init(d_full + i, 1);
+            mbar_init(d_empty + i, C::NCW);
+        }
+        mbar_init(mq_full, 1);
+        mbar_init(mq_empty, 1);
+        for (int i = 0; i < C::NBUF; ++i) {
+            mbar_init(tm_full + i, 1);
+            mbar_init(tm_empty + i, 4 * C::HG);  // the warps of the group's heads
+        }
+        for (int i = 0; i < C::NK; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(k_empty + i, C::HC);  // the head warps of the quarter
+        }
+        for (int i = 0; i < C::NV; ++i) {
+            mbar_init(v_full + i, 1);
+            mbar_init(v_empty + i, 1);  // V GEMM commit
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    TileWalker wk;
+    wk.init(p.P, p.B, p.G, blockIdx.x, C::PARTS);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ M_q, Phi, c^K loads
+        if (elect_one()) {
+            prefetch_tensormap(&lat_map);
+            const uint64_t pol_stream = policy_evict_first();
+            const uint64_t pol_keep = policy_evict_last();
+            uint32_t kk_n = 0, phi_n = 0, mq_n = 0;
+            int prev_key = -1;
+            bool ok = true;
+            for (; wk.valid() && ok; wk.next()) {
+                const int key = wk.key();
+                if (key != prev_key) {
+                    if (mq_n > 0 && !(ok = mbar_wait(mq_empty, (mq_n - 1) & 1, p.status, kFlagTimeout, 21))) break;
+                    mbar_expect_tx(mq_full, C::MQ_BYTES);
+                    const uint8_t* src = p.mq + (size_t(wk.p) * p.B + wk.b) * C::MQ_BYTES;
+                    for (int off = 0; off < C::MQ_BYTES; off += 32768) {
+                        const int n = C::MQ_BYTES - off < 32768 ? C::MQ_BYTES - off : 32768;
+                        bulk_g2s(mq_s + off, src + off, n, mq_full, pol_keep);
+                    }
+                    ++mq_n;
+                    prev_key = key;
+                }
+                {
+                    const uint32_t pb = phi_n & 1, pr = phi_n >> 1;
+                    if (pr > 0 && !(ok = mbar_wait(phi_empty + pb, (pr - 1) & 1, p.status, kFlagTimeout, 22))) break;
+                    mbar_expect_tx(phi_full + pb, C::PHI_BYTES);
+                    bulk_g2s(phi_s + pb * C::PHI_BYTES, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES,
+                             phi_full + pb, pol_keep);
+                    ++phi_n;
+                }
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t slot = kk_n % C::NK, round = kk_n / C::NK;
+                    if (round > 0 && !(ok = mbar_wait(k_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 23)))
+                        break;
+                    mbar_expect_tx(k_full + slot, C::K_SLOT);
+                    tma_load_4d(k_s + size_t(slot) * C::K_SLOT, &lat_map, 0, 0, wk.t * kTile + q * C::QTOK, wk.b,
+                                k_full + slot, pol_stream);
+                    __threadfence_block();  // the armed barrier phase precedes the published round
+                    k_issued[slot] = round + 1;
+                    ++kk_n;
+                }
+            }
+            // no copy may still be in flight when the CTA exits
+            wait_last_phases(k_full, C::NK, kk_n, p.status, 24);
+            wait_last_phases(phi_full, 2, phi_n, p.status, 25);
+            if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 26);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ c^V loads
+        if (elect_one()) {
+            const uint64_t pol_stream = policy_evict_first();
+            uint32_t vk_n = 0;
+            bool ok = true;
+            for (; wk.valid() && ok; wk.next()) {
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t slot = vk_n % C::NV, round = vk_n / C::NV;
+                    if (round > 0 && !(ok = mbar_wait(v_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 27)))
+                        break;
+                    mbar_expect_tx(v_full + slot, C::V_SLOT);
+#pragma unroll
+                    for (int pn = 0; pn < C::V_PANELS; ++pn)
+                        tma_load_4d(v_s + size_t(slot) * C::V_SLOT + pn * C::PANEL, &lat_map, C::RK + 64 * pn, 0,
+                                    wk.t * kTile + q * C::QTOK, wk.b, v_full + slot, pol_stream);
+                    __threadfence_block();
+                    v_issued[slot] = round + 1;
+                    ++vk_n;
+                }
+            }
+            wait_last_phases(v_full, C::NV, vk_n, p.status, 28);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t phi_n = 0, mq_n = 0, mq_commits = 0, tile_n = 0, v_commits = 0, v_next = 0;
+            int prev_key = -1;
+            bool ok = true;
+            const uint32_t phi_addr = smem_u32(phi_s), mq_addr = smem_u32(mq_s);
+            const uint32_t p_addr = smem_u32(p_s), v_addr = smem_u32(v_s);
+            // V GEMM of tile n: D[pb] = sum over its 8 sixteen-token steps of (C^V)^T . P
+            auto issue_v = [&](uint32_t n) -> bool {
+                const uint32_t pb = n & 1, use = n >> 1;
+                if (!mbar_wait(p_full + pb, use & 1, p.status, kFlagTimeout, 29)) return false;
+                if (use > 0 && !mbar_wait(d_empty + pb, (use - 1) & 1, p.status, kFlagTimeout, 30)) return false;
+                const uint32_t d_tmem = tmem_base + C::VCOL + pb * C::VN;
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t vs = n * 4 + q, slot = vs % C::NV;
+                    if (!mbar_wait(v_full + slot, (vs / C::NV) & 1, p.status, kFlagTimeout, 31)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const int kk = 2 * q + k2;  // sixteen-token step of the tile
+                        const uint64_t ad = sw128_mnmajor_desc(v_addr + slot * C::V_SLOT + k2 * (16 * 128),
+                                                               C::PANEL, 1024);
+                        const uint64_t bd = sw128_kmajor_desc(p_addr + pb * C::P_BYTES +
+                                                              uint32_t(kk >> 2) * (C::VN * 128) + uint32_t(kk & 3) * 32);
+                        mma_f16_ss(d_tmem, ad, bd, C::IDESC_V, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(v_empty + slot);
+                    ++v_commits;
+                }
+                mma_commit(d_full + pb);
+                return true;
+            };
+            // V GEMMs of every tile before `end` not issued yet
+            auto issue_v_upto = [&](uint32_t end) -> bool {
+                for (; v_next < end; ++v_next)
+                    if (!issue_v(v_next)) return false;
+                return true;
+            };
+            for (; wk.valid() && ok; wk.next(), ++tile_n) {
+                const int key = wk.key();
+                if (key != prev_key) {
+                    if (prev_key != -1) {
+                        mma_commit(mq_empty);
+                        ++mq_commits;
+                    }
+                    // the compute warps close the previous sequence with its last V GEMM: issue
+                    // it before waiting for the next M_q image
+                    if (!(ok = issue_v_upto(tile_n))) break;
+                    if (!(ok = mbar_wait(mq_full, mq_n & 1, p.status, kFlagTimeout, 32))) break;
+                    ++mq_n;
+                    prev_key = key;
+                }
+                const uint32_t pb = phi_n & 1;
+                if (!(ok = mbar_wait(phi_full + pb, (phi_n >> 1) & 1, p.status, kFlagTimeout, 33))) break;
+                ++phi_n;
+                tc_fence_after();
+                const uint32_t phi_buf = phi_addr + pb * C::PHI_BYTES;
+                for (int g = 0; g < C::GPC && ok; ++g) {
+                    const uint32_t gi = tile_n * C::GPC + g;
+                    const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
+                    if (use > 0 && !(ok = mbar_wait(tm_empty + buf, (use - 1) & 1, p.status, kFlagTimeout, 34))) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + buf * C::BUF_COLS;
+#pragma unroll
+                    for (int kk = 0; kk < C::DH / 16; ++kk) {
+                        const uint32_t koff = uint32_t(kk & 3) * 32;
+                        const uint64_t ad = sw128_kmajor_desc(phi_buf + uint32_t(kk >> 2) * (kTile * 128) + koff);
+                        const uint64_t bd = sw128_kmajor_desc(mq_addr + g * C::MQ_GROUP_BYTES +
+                                                              uint32_t(kk >> 2) * (C::NG * 128) + koff);
+                        mma_f16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(tm_full + buf);
+                }
+                if (!ok) break;
+                mma_commit(phi_empty + pb);
+                ok = issue_v_upto(tile_n);  // the previous tile's P is complete once its scores are
+            }
+            if (ok) ok = issue_v_upto(tile_n);
+            if (prev_key != -1) {
+                mma_commit(mq_empty);
+                ++mq_commits;
+            }
+            // the commits' arrivals land in shared memory: see them complete before the CTA exits
+            wait_last_phases(phi_empty, 2, phi_n, p.status, 35);
+            wait_last_phases(v_empty, C::NV, v_commits, p.status, 36);
+            if (mq_commits > 0) mbar_wait(mq_empty, (mq_commits - 1) & 1, p.status, kFlagTimeout, 37);
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int cw = warp - 3;
+        const int qd = warp & 3;            // TMEM lane quarter = token rows [32 qd, 32 qd + 32)
+        const int hf = cw >> 2;             // head of the CTA item
+        const int g = hf / C::HG, hg = hf % C::HG;
+        const uint32_t lane_addr = uint32_t(32 * qd) << 16;
+        const int pcol = hf * 4 + qd;       // this warp's column of P
+        const uint32_t p_off = sw128_offset(pcol, 32 * qd + lane, C::VN);
+
+        float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float isc = 0.f;
+        int len = 0;
+        uint32_t tile_n = 0;
+        int prev_key = -1;
+        long long prev_id = 0;
+        bool ok = true, pending = false;
+
+        auto sync_ok = [&](bool w) { ok = __all_sync(0xffffffffu, w) && ok; };
+
+        // V GEMM result of tile n: acc_{q,h} = alpha_{q,h} acc_{q,h} + D[:, (h, q)] for the
+        // r_v dimensions of this lane quarter and every source quarter q
+        auto accumulate = [&](uint32_t n) {
+            const uint32_t pb = n & 1, use = n >> 1;
+            // p_full: the alpha values, written before its arrivals; d_full: the GEMM
+            bool w = mbar_wait(p_full + pb, use & 1, p.status, kFlagTimeout, 38);
+            w = w && mbar_wait(d_full + pb, use & 1, p.status, kFlagTimeout, 39);
+            sync_ok(w);
+            tc_fence_after();
+            float d[4];
+            tmem_ld<4>(tmem_base + lane_addr + C::VCOL + pb * C::VN + hf * 4, d);
+            tmem_wait_ld();
+            const float* al = alpha_s + pb * (4 * C::HC) + hf;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fmaf(acc[q], al[q * C::HC], d[q]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(d_empty + pb);
+        };
+
+        auto flush = [&](long long id) {
+            const size_t rl = C::RV + 2;
+            float* set = p.records + size_t(id) * 4 * C::HC * rl;  // record (q, h) at (q * HC + h) * rl
+            const float lsum = warp_sum(l);
+            if (lane == 0) {
+                float* own = set + (size_t(qd) * C::HC + hf) * rl;
+                own[0] = (m == -INFINITY) ? -INFINITY : m * kLn2;
+                own[1] = lsum;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) set[(size_t(q) * C::HC + hf) * rl + 2 + 32 * qd + lane] = acc[q];
+        };
+
+        for (; wk.valid() && ok; wk.next(), ++tile_n) {
+            const int key = wk.key();
+            if (key != prev_key) {
+                if (pending) {
+                    accumulate(tile_n - 1);
+                    pending = false;
+                }
+                if (prev_key != -1) flush(prev_id);
+                m = -INFINITY;
+                l = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[q] = 0.f;
+                prev_key = key;
+                prev_id = wk.record_id();
+                isc = __ldg(p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC + hf);
+                len = __ldg(p.lens + wk.b);
+            }
+            const int valid = min(kTile, len - wk.t * kTile);
+            const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this quarter
+            const bool row_ok = lane < nv;
+
+            // ---- score: s = c^K . G + bias, G from TMEM, c^K from this quarter's slot
+            const uint32_t gi = tile_n * C::GPC + g;
+            const uint32_t buf = gi % C::NBUF;
+            sync_ok(mbar_wait(tm_full + buf, (gi / C::NBUF) & 1, p.status, kFlagTimeout, 40));
+            const uint32_t ks = tile_n * 4 + qd, kslot = ks % C::NK;
+            {
+                bool w = true;
+                if (lane == 0) {
+                    w = ok && wait_issued(k_issued + kslot, ks / C::NK + 1, p.status, kFlagTimeout, 41);
+                    w = w && mbar_wait(k_full + kslot, (ks / C::NK) & 1, p.status, kFlagTimeout, 42);
+                }
+                ok = __shfl_sync(0xffffffffu, w, 0) && ok;
+                __syncwarp();
+            }
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
+            const uint8_t* krow = k_s + size_t(kslot) * C::K_SLOT + lane * 128;
+            float bias;
+            tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
+            uint64_t s01 = 0, s23 = 0;
+#pragma unroll
+            for (int a0 = 0; a0 < C::RK; a0 += 16) {
+                float gv[16];
+                tmem_ld<16>(tcol + hg * C::RK + a0, &gv[0]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int chunk = (a0 >> 3) + c;  // 16-byte chunk of the row, before the swizzle
+                    const uint4 u = *reinterpret_cast<const uint4*>(krow + ((chunk ^ (lane & 7)) << 4));
+                    const int c0 = 8 * c;
+                    s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[c0 + 0], gv[c0 + 1]), s01);
+                    s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[c0 + 2], gv[c0 + 3]), s23);
+                    s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[c0 + 4], gv[c0 + 5]), s01);
+                    s23 = f2_fma(bf16x2_to_f2(u.w), f2_pack(gv[c0 + 6], gv[c0 + 7]), s23);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(tm_empty + buf);
+                mbar_arrive(k_empty + kslot);
+            }
+            const float2 sp = f2_unpack(s01), sq = f2_unpack(s23);
+            const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * isc : -INFINITY;
+
+            // ---- online softmax in base 2; p is rounded to bf16 for the V GEMM and l sums
+            // the rounded values, so that numerator and denominator see the same weights
+            const float m_new = fmaxf(m, warp_max(s2));
+            const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m - m_new);
+            const float pj = row_ok ? fast_exp2(s2 - m_new) : 0.f;
+            const __nv_bfloat16 pbf = __float2bfloat16_rn(pj);
+            const uint16_t pbits = *reinterpret_cast<const uint16_t*>(&pbf);
+            l = fmaf(l, alpha, bf16_to_f32(pbits));
+            m = m_new;
+
+            // ---- P and alpha into buffer tile_n & 1, last used by tile n - 2, whose V GEMM
+            // and readers must be done with it
+            const uint32_t pb = tile_n & 1;
+            if (tile_n >= 2) sync_ok(mbar_wait(d_empty + pb, ((tile_n >> 1) - 1) & 1, p.status, kFlagTimeout, 43));
+            *reinterpret_cast<uint16_t*>(p_s + pb * C::P_BYTES + p_off) = pbits;
+            if (lane == 0) alpha_s[pb * (4 * C::HC) + qd * C::HC + hf] = alpha;
+            if (hf == 0 && nv < 32) {
+                // rows past the context may hold any bits, and 0 * NaN is not 0: clear them in
+                // the c^V slot before the V GEMM reads it
+                const uint32_t vs = tile_n * 4 + qd, vslot = vs % C::NV;
+                bool w = true;
+                if (lane == 0) {
+                    w = ok && wait_issued(v_issued + vslot, vs / C::NV + 1, p.status, kFlagTimeout, 44);
+                    w = w && mbar_wait(v_full + vslot, (vs / C::NV) & 1, p.status, kFlagTimeout, 45);
+                }
+                ok = __shfl_sync(0xffffffffu, w, 0) && ok;
+                __syncwarp();
+                if (lane >= nv) {
+                    uint8_t* row = v_s + size_t(vslot) * C::V_SLOT + lane * 128;
+#pragma unroll
+                    for (int pn = 0; pn < C::V_PANELS; ++pn)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(row + pn * C::PANEL + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full + pb);
+
+            // ---- the previous tile's V GEMM, complete by now or shortly
+            if (pending) accumulate(tile_n - 1);
+            pending = true;
+        }
+        if (pending && ok) accumulate(tile_n - 1);
+        if (prev_key != -1) flush(prev_id);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}

@@ -193,6 +193,36 @@ def test_2d_matches_oracle(c):
     lib.close()
 
 
+@pytest.mark.parametrize("variant,rk,rv", [(0, 16, 32), (0, 96, 160), (1, 64, 128)])
+def test_rows_past_the_context_may_hold_nan(variant, rk, rv):
+    """Store rows at or beyond a sequence's length are outside the attention [LLA §3 eq. (3)
+    sums over the cached tokens only]: a quiet-NaN pattern there must not reach the output."""
+    B, N, D, T, H, d = 3, 300, 1, 2, 16, 128
+    lens = [300, 77, 130]
+    tag = f"nan_tail/{variant}/{rk}"
+    cfg = dict(D=D, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0, mu_var=0.1)
+    codec = rounded_codec(syn.seeded_codec(cfg, tag))
+    head = () if variant == 1 else (H,)
+    cK = syn.round_bf16(syn.gaussian(tag + "/cK", (B, D, N) + head + (rk,)))
+    cV = syn.round_bf16(syn.gaussian(tag + "/cV", (B, D, N) + head + (rv,)))
+    q = syn.round_f32(syn.gaussian(tag + "/q", (B, H, d)))
+    bits = to_bf16_bits(np.concatenate([cK, cV], -1))
+    for b, n in enumerate(lens):
+        bits[b, :, n:] = 0x7FC0  # bf16 quiet NaN
+    lib = make_lib_codec(lla, dict(D=D, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0,
+                                   max_pos=N + 4), codec)
+    scale = 1 / math.sqrt(d)
+    ref = oracle_decode(codec, cfg, cK[:, 0], cV[:, 0], q, 0, 1, lens, lens, scale)
+    impls = [lla.IMPL_SIMT] + ([lla.IMPL_TC] if _tc_supported(lib, B, N) else [])
+    assert lla.IMPL_TC in impls
+    for impl in impls:
+        got, flags = _run(lib, bits, B, N, 0, 1, q, lens, lens, scale, impl=impl)
+        assert flags == 0
+        assert np.isfinite(got).all(), f"impl {impl}"
+        assert_close(got, ref, f"nan tail impl {impl}")
+    lib.close()
+
+
 # ---------------------------------------------------------------------------------------------
 # range flags
 # ---------------------------------------------------------------------------------------------
