@@ -139,7 +139,7 @@ struct TileWalker {
     const int32_t* P;
     int B, parts;
     long long x, x1, total;
-    int p, gi, b, t;
+    int p, gi, b, t, nt;  // nt: tiles of sequence b (kept in a register, not re-read per tile)
     __device__ void init(const int32_t* P_, int B_, int G, int cta, int parts_) {
         P = P_;
         B = B_;
@@ -163,6 +163,7 @@ struct TileWalker {
         }
         b = lo;
         t = int(x - P[b]);
+        nt = P[b + 1] - P[b];
     }
     __device__ bool valid() const { return x < x1; }
     __device__ int key() const { return b; }  // M_q image and record set change with the sequence
@@ -171,9 +172,10 @@ struct TileWalker {
         ++x;
         if (x >= x1) return;
         ++t;
-        while (t >= P[b + 1] - P[b]) {
+        while (t >= nt) {
             t = 0;
             ++b;
+            nt = P[b + 1] - P[b];
         }
     }
 };
@@ -359,6 +361,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 
         float m[C::HPW], l[C::HPW], acc[C::HPW][C::VPL];
         const float* isc_row = p.inv_scale;  // per-(b, h) score scale, re-read from L1 when needed
+        int len = 0;                         // clamped length of the current sequence
         uint32_t gi = 0, tile_n = 0;
         int prev_key = -1;
         long long prev_id = 0;
@@ -415,8 +418,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 prev_key = key;
                 prev_id = wk.record_id();
                 isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
+                len = __ldg(p.lens + wk.b);
             }
-            const int valid = min(kTile, p.lens[wk.b] - wk.t * kTile);
+            const int valid = min(kTile, len - wk.t * kTile);
             const bool row_ok = row < valid;
             const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this warp
 

@@ -46,7 +46,8 @@ struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
     static constexpr int NV_RAW = (kSmemLimit - FIXED - NK * K_SLOT) / V_SLOT;
     static constexpr int NV = NV_RAW > 16 ? 16 : NV_RAW;
     static constexpr int SMEM = FIXED + NK * K_SLOT + NV * V_SLOT;
-    static constexpr int NCW = 4 * HC;                  // one compute warp per (quarter, head)
+    static constexpr int HPW = HG;                      // heads per compute warp: one TMEM group
+    static constexpr int NCW = 4 * (HC / HPW);          // one compute warp per (quarter, head group)
     static constexpr int THREADS = 32 * (3 + NCW);
     static constexpr int TMEM_COLS = 512;
     static constexpr int NBUF = 3;                      // score accumulator ring
@@ -97,8 +98,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     uint64_t* v_full = k_empty + C::NK;       // [NV]
     uint64_t* v_empty = v_full + C::NV;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_empty + C::NV);
-    // loads issued per slot (a consumer first waits for its round to be issued, so that a
-    // parity wait cannot match an earlier round of the slot)
+    // loads issued per slot (a compute warp first waits for its round to be issued, so that
+    // its parity wait cannot match an earlier round of the slot)
     volatile uint32_t* k_issued = tmem_holder + 1;
     volatile uint32_t* v_issued = k_issued + C::NK;
     float* alpha_s = reinterpret_cast<float*>(tmem_holder + 64);  // [2][4 quarters][HC]
@@ -122,11 +123,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         mbar_init(mq_empty, 1);
         for (int i = 0; i < C::NBUF; ++i) {
             mbar_init(tm_full + i, 1);
-            mbar_init(tm_empty + i, 4 * C::HG);  // the warps of the group's heads
+            mbar_init(tm_empty + i, 4);  // the group's warp of each quarter
         }
         for (int i = 0; i < C::NK; ++i) {
             mbar_init(k_full + i, 1);
-            mbar_init(k_empty + i, C::HC);  // the head warps of the quarter
+            mbar_init(k_empty + i, C::HC / C::HPW);  // the group warps of the quarter
         }
         for (int i = 0; i < C::NV; ++i) {
             mbar_init(v_full + i, 1);
@@ -306,16 +307,19 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         }
     } else {
         // ------------------------------------------------------------ compute warps
+        // one warp per (TMEM lane quarter, head group): the HPW heads of a group share the
+        // warp's c^K loads and conversions, its waits and its barrier arrivals
+        constexpr int HPW = C::HPW;
         const int cw = warp - 3;
         const int qd = warp & 3;            // TMEM lane quarter = token rows [32 qd, 32 qd + 32)
-        const int hf = cw >> 2;             // head of the CTA item
-        const int g = hf / C::HG, hg = hf % C::HG;
+        const int g = cw >> 2;              // head group of the CTA item
+        const int hf0 = g * HPW;            // first head of the item in this warp
         const uint32_t lane_addr = uint32_t(32 * qd) << 16;
-        const int pcol = hf * 4 + qd;       // this warp's column of P
-        const uint32_t p_off = sw128_offset(pcol, 32 * qd + lane, C::VN);
 
-        float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-        float isc = 0.f;
+        float m[HPW], l[HPW], acc[HPW][4], isc[HPW];
+        uint32_t p_off[HPW];  // this lane's entry of P, per head
+#pragma unroll
+        for (int hh = 0; hh < HPW; ++hh) p_off[hh] = sw128_offset((hf0 + hh) * 4 + qd, 32 * qd + lane, C::VN);
         int len = 0;
         uint32_t tile_n = 0;
         int prev_key = -1;
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         auto sync_ok = [&](bool w) { ok = __all_sync(0xffffffffu, w) && ok; };
 
         // V GEMM result of tile n: acc_{q,h} = alpha_{q,h} acc_{q,h} + D[:, (h, q)] for the
-        // r_v dimensions of this lane quarter and every source quarter q
+        // r_v dimensions of this lane quarter, every source quarter q and this warp's heads
         auto accumulate = [&](uint32_t n) {
             const uint32_t pb = n & 1, use = n >> 1;
             // p_full: the alpha values, written before its arrivals; d_full: the GEMM
@@ -333,12 +337,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             w = w && mbar_wait(d_full + pb, use & 1, p.status, kFlagTimeout, 39);
             sync_ok(w);
             tc_fence_after();
-            float d[4];
-            tmem_ld<4>(tmem_base + lane_addr + C::VCOL + pb * C::VN + hf * 4, d);
+            float d[4 * HPW];
+            tmem_ld<4 * HPW>(tmem_base + lane_addr + C::VCOL + pb * C::VN + hf0 * 4, d);
             tmem_wait_ld();
-            const float* al = alpha_s + pb * (4 * C::HC) + hf;
+            const float* al = alpha_s + pb * (4 * C::HC) + hf0;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] = fmaf(acc[q], al[q * C::HC], d[q]);
+            for (int hh = 0; hh < HPW; ++hh)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[hh][q] = fmaf(acc[hh][q], al[q * C::HC + hh], d[hh * 4 + q]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(d_empty + pb);
@@ -347,14 +353,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         auto flush = [&](long long id) {
             const size_t rl = C::RV + 2;
             float* set = p.records + size_t(id) * 4 * C::HC * rl;  // record (q, h) at (q * HC + h) * rl
-            const float lsum = warp_sum(l);
-            if (lane == 0) {
-                float* own = set + (size_t(qd) * C::HC + hf) * rl;
-                own[0] = (m == -INFINITY) ? -INFINITY : m * kLn2;
-                own[1] = lsum;
-            }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) set[(size_t(q) * C::HC + hf) * rl + 2 + 32 * qd + lane] = acc[q];
+            for (int hh = 0; hh < HPW; ++hh) {
+                const int hf = hf0 + hh;
+                const float lsum = warp_sum(l[hh]);
+                if (lane == 0) {
+                    float* own = set + (size_t(qd) * C::HC + hf) * rl;
+                    own[0] = (m[hh] == -INFINITY) ? -INFINITY : m[hh] * kLn2;
+                    own[1] = lsum;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) set[(size_t(q) * C::HC + hf) * rl + 2 + 32 * qd + lane] = acc[hh][q];
+            }
         };
 
         for (; wk.valid() && ok; wk.next(), ++tile_n) {
@@ -365,20 +375,23 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     pending = false;
                 }
                 if (prev_key != -1) flush(prev_id);
-                m = -INFINITY;
-                l = 0.f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q] = 0.f;
+                for (int hh = 0; hh < HPW; ++hh) {
+                    m[hh] = -INFINITY;
+                    l[hh] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[hh][q] = 0.f;
+                    isc[hh] = __ldg(p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC + hf0 + hh);
+                }
                 prev_key = key;
                 prev_id = wk.record_id();
-                isc = __ldg(p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC + hf);
                 len = __ldg(p.lens + wk.b);
             }
             const int valid = min(kTile, len - wk.t * kTile);
             const int nv = max(0, min(32, valid - 32 * qd));  // valid rows of this quarter
             const bool row_ok = lane < nv;
 
-            // ---- score: s = c^K . G + bias, G from TMEM, c^K from this quarter's slot
+            // ---- scores of the group's heads: s = c^K . G + bias, G from TMEM
             const uint32_t gi = tile_n * C::GPC + g;
             const uint32_t buf = gi % C::NBUF;
             sync_ok(mbar_wait(tm_full + buf, (gi / C::NBUF) & 1, p.status, kFlagTimeout, 40));
@@ -396,23 +409,41 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             tc_fence_after();
             const uint32_t tcol = tmem_base + lane_addr + buf * C::BUF_COLS;
             const uint8_t* krow = k_s + size_t(kslot) * C::K_SLOT + lane * 128;
-            float bias;
-            tmem_ld<1>(tcol + C::HG * C::RK + hg, &bias);
-            uint64_t s01 = 0, s23 = 0;
+            float bias[HPW];
 #pragma unroll
-            for (int a0 = 0; a0 < C::RK; a0 += 16) {
-                float gv[16];
-                tmem_ld<16>(tcol + hg * C::RK + a0, &gv[0]);
-                tmem_wait_ld();
+            for (int hh = 0; hh < HPW; ++hh) tmem_ld<1>(tcol + C::HG * C::RK + hh, &bias[hh]);
+            uint64_t s01[HPW], s23[HPW];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int chunk = (a0 >> 3) + c;  // 16-byte chunk of the row, before the swizzle
-                    const uint4 u = *reinterpret_cast<const uint4*>(krow + ((chunk ^ (lane & 7)) << 4));
-                    const int c0 = 8 * c;
-                    s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[c0 + 0], gv[c0 + 1]), s01);
-                    s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[c0 + 2], gv[c0 + 3]), s23);
-                    s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[c0 + 4], gv[c0 + 5]), s01);
-                    s23 = f2_fma(bf16x2_to_f2(u.w), f2_pack(gv[c0 + 6], gv[c0 + 7]), s23);
+            for (int hh = 0; hh < HPW; ++hh) s01[hh] = s23[hh] = 0;
+            // 16 latent dimensions at a time, the next 16 columns of G in flight while the
+            // current ones are used; the c^K words are converted once for all heads
+            float ga[HPW][16], gb[HPW][16];
+#pragma unroll
+            for (int hh = 0; hh < HPW; ++hh) tmem_ld<16>(tcol + hh * C::RK, ga[hh]);
+#pragma unroll
+            for (int hh = 0; hh < HPW; ++hh) tmem_wait_ld_regs16(ga[hh]);
+#pragma unroll
+            for (int a16 = 0; a16 < C::RK / 16; ++a16) {
+                float(*cur)[16] = (a16 & 1) ? gb : ga;
+                float(*nxt)[16] = (a16 & 1) ? ga : gb;
+                if (a16 + 1 < C::RK / 16) {
+#pragma unroll
+                    for (int hh = 0; hh < HPW; ++hh) tmem_ld<16>(tcol + hh * C::RK + 16 * (a16 + 1), nxt[hh]);
+                }
+                const uint4 u0 = *reinterpret_cast<const uint4*>(krow + (((2 * a16) ^ (lane & 7)) << 4));
+                const uint4 u1 = *reinterpret_cast<const uint4*>(krow + (((2 * a16 + 1) ^ (lane & 7)) << 4));
+                const uint64_t c2[8] = {bf16x2_to_f2(u0.x), bf16x2_to_f2(u0.y), bf16x2_to_f2(u0.z), bf16x2_to_f2(u0.w),
+                                        bf16x2_to_f2(u1.x), bf16x2_to_f2(u1.y), bf16x2_to_f2(u1.z), bf16x2_to_f2(u1.w)};
+#pragma unroll
+                for (int hh = 0; hh < HPW; ++hh)
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        s01[hh] = f2_fma(c2[e], f2_pack(cur[hh][2 * e], cur[hh][2 * e + 1]), s01[hh]);
+                        s23[hh] = f2_fma(c2[e + 1], f2_pack(cur[hh][2 * e + 2], cur[hh][2 * e + 3]), s23[hh]);
+                    }
+                if (a16 + 1 < C::RK / 16) {
+#pragma unroll
+                    for (int hh = 0; hh < HPW; ++hh) tmem_wait_ld_regs16(nxt[hh]);
                 }
             }
             tc_fence_before();
@@ -421,26 +452,37 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 mbar_arrive(tm_empty + buf);
                 mbar_arrive(k_empty + kslot);
             }
-            const float2 sp = f2_unpack(s01), sq = f2_unpack(s23);
-            const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * isc : -INFINITY;
 
             // ---- online softmax in base 2; p is rounded to bf16 for the V GEMM and l sums
             // the rounded values, so that numerator and denominator see the same weights
-            const float m_new = fmaxf(m, warp_max(s2));
-            const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m - m_new);
-            const float pj = row_ok ? fast_exp2(s2 - m_new) : 0.f;
-            const __nv_bfloat16 pbf = __float2bfloat16_rn(pj);
-            const uint16_t pbits = *reinterpret_cast<const uint16_t*>(&pbf);
-            l = fmaf(l, alpha, bf16_to_f32(pbits));
-            m = m_new;
-
-            // ---- P and alpha into buffer tile_n & 1, last used by tile n - 2, whose V GEMM
-            // and readers must be done with it
+            float s2[HPW], mx[HPW];
+#pragma unroll
+            for (int hh = 0; hh < HPW; ++hh) {
+                const float2 sp = f2_unpack(s01[hh]), sq = f2_unpack(s23[hh]);
+                s2[hh] = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias[hh]) * isc[hh] : -INFINITY;
+                mx[hh] = s2[hh];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int hh = 0; hh < HPW; ++hh) mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], o));
             const uint32_t pb = tile_n & 1;
+            // P and alpha go to buffer tile_n & 1, last used by tile n - 2, whose V GEMM and
+            // readers must be done with it
             if (tile_n >= 2) sync_ok(mbar_wait(d_empty + pb, ((tile_n >> 1) - 1) & 1, p.status, kFlagTimeout, 43));
-            *reinterpret_cast<uint16_t*>(p_s + pb * C::P_BYTES + p_off) = pbits;
-            if (lane == 0) alpha_s[pb * (4 * C::HC) + qd * C::HC + hf] = alpha;
-            if (hf == 0 && nv < 32) {
+#pragma unroll
+            for (int hh = 0; hh < HPW; ++hh) {
+                const float m_new = fmaxf(m[hh], mx[hh]);
+                const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m[hh] - m_new);
+                const float pj = row_ok ? fast_exp2(s2[hh] - m_new) : 0.f;
+                const __nv_bfloat16 pbf = __float2bfloat16_rn(pj);
+                const uint16_t pbits = *reinterpret_cast<const uint16_t*>(&pbf);
+                l[hh] = fmaf(l[hh], alpha, bf16_to_f32(pbits));
+                m[hh] = m_new;
+                *reinterpret_cast<uint16_t*>(p_s + pb * C::P_BYTES + p_off[hh]) = pbits;
+                if (lane == 0) alpha_s[pb * (4 * C::HC) + qd * C::HC + hf0 + hh] = alpha;
+            }
+            if (g == 0 && nv < 32) {
                 // rows past the context may hold any bits, and 0 * NaN is not 0: clear them in
                 // the c^V slot before the V GEMM reads it
                 const uint32_t vs = tile_n * 4 + qd, vslot = vs % C::NV;
