@@ -58,7 +58,7 @@ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // Head grouping shared by both kernels: which heads share one score GEMM (a TMEM group,
 // N <= 256 columns), how many groups stay resident per CTA (their M_q images), and so how
 // many CTAs ("parts") split the heads of a tile.
-template <int DH_, int RK_, int RV_, int H_>
+template <int DH_, int RK_, int RV_, int H_, int GPC_CAP = 8>
 struct HeadGroups {
     static constexpr int DH = DH_, RK = RK_, RV = RV_, H = H_;
     // heads per TMEM group: as many as fit N <= 256 (even, dividing H)
@@ -68,7 +68,8 @@ struct HeadGroups {
     static constexpr int NG = round_up(HG * RK + HG, 16);
     static constexpr int MQ_GROUP_BYTES = NG * DH * 2;
     static constexpr int GPC_MAX = (110 * 1024) / MQ_GROUP_BYTES;  // resident M_q budget ~110 KB
-    static constexpr int GPC = (H / HG) <= GPC_MAX ? (H / HG) : ((H / HG) % 2 == 0 && GPC_MAX >= 2 ? 2 : 1);
+    static constexpr int GPC_FIT = (H / HG) <= GPC_MAX ? (H / HG) : ((H / HG) % 2 == 0 && GPC_MAX >= 2 ? 2 : 1);
+    static constexpr int GPC = GPC_FIT < GPC_CAP ? GPC_FIT : GPC_CAP;
     static constexpr int HC = HG * GPC;  // heads per CTA work item
     static constexpr int PARTS = H / HC;
     static constexpr int MQ_BYTES = GPC * MQ_GROUP_BYTES;
@@ -78,10 +79,13 @@ struct HeadGroups {
     static_assert(H % HC == 0 && HG % 2 == 0, "head split");
 };
 
-// Per-head latent rows (one row of r_k + r_v per (token, head)).
-template <int DH_, int RK_, int RV_, int H_>
-struct Cfg : HeadGroups<DH_, RK_, RV_, H_> {
-    using HG_ = HeadGroups<DH_, RK_, RV_, H_>;
+// Per-head latent rows (one row of r_k + r_v per (token, head)).  Wide rows (512 B and up)
+// make a 32-token stage of one head 16 KB: such codecs keep one head group resident (a
+// deeper stage ring) and give each lane quarter one compute warp, which walks the heads of
+// the item in turn, so that at most four stages are being read while the rest prefetch.
+template <int DH_, int RK_, int RV_, int H_, bool WIDE = (RK_ + RV_) * 2 >= 512>
+struct Cfg : HeadGroups<DH_, RK_, RV_, H_, WIDE ? 1 : 8> {
+    using HG_ = HeadGroups<DH_, RK_, RV_, H_, WIDE ? 1 : 8>;
     using HG_::DH, HG_::RK, HG_::RV, HG_::H, HG_::HG, HG_::NG, HG_::HC, HG_::MQ_BYTES, HG_::PHI_BYTES;
     static constexpr bool TWO_D = false;
     static constexpr int ROW = RK + RV;
@@ -94,7 +98,7 @@ struct Cfg : HeadGroups<DH_, RK_, RV_, H_> {
     static constexpr int NST = NST_RAW > 32 ? 32 : NST_RAW;
     static constexpr int SMEM = FIXED + NST * STAGE_BYTES;
     // compute warps: WPQ per TMEM lane quarter, each taking HG / WPQ heads of every group
-    static constexpr int WPQ = HG >= 4 ? 4 : HG;
+    static constexpr int WPQ = WIDE ? 1 : (HG >= 4 ? 4 : HG);
     static constexpr int NCW = 4 * WPQ;
     static constexpr int THREADS = 32 * (2 + NCW);
     static constexpr int HPW = HC / WPQ;  // heads per compute warp
@@ -109,7 +113,7 @@ struct Cfg : HeadGroups<DH_, RK_, RV_, H_> {
     static constexpr bool VQUAD = (RV == 32 || RV == 64 || RV == 128);
     static constexpr int VAL = VQUAD ? RV / 4 : 32;          // lanes along the latent dimension
     static constexpr int VTL = 32 / VAL;                      // token sub-lanes
-    static constexpr int VPL = VQUAD ? 4 : RV / 32;           // accumulators per lane per head
+    static constexpr int VPL = VQUAD ? 4 : RV / 16;           // accumulators per lane per head
     static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
     static_assert(HC % WPQ == 0, "head split");
     static_assert(NG <= BUF_COLS, "TMEM buffer");
@@ -398,8 +402,19 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 #pragma unroll
                         for (int v = 0; v < 4; ++v) rec[2 + 4 * lane + v] = a[v];
                 } else {
+                    // lane l16 < 16 holds words l16 + 16 k (k < NW) of the even tokens; lane l16 + 16
+                    // holds the odd tokens' words in rotated order: its slot k - 1 is word l16 + 16 k
+                    constexpr int NW = C::RV / 32;
 #pragma unroll
-                    for (int v = 0; v < C::VPL; ++v) rec[2 + lane + 32 * v] = a[v];
+                    for (int k = 0; k < NW; ++k) {
+                        const int ko = k == 0 ? NW - 1 : k - 1;
+                        const float o0 = __shfl_down_sync(0xffffffffu, acc[hw][2 * ko], 16);
+                        const float o1 = __shfl_down_sync(0xffffffffu, acc[hw][2 * ko + 1], 16);
+                        if (lane < 16) {
+                            rec[2 + 2 * (lane + 16 * k)] = acc[hw][2 * k] + o0;
+                            rec[2 + 2 * (lane + 16 * k) + 1] = acc[hw][2 * k + 1] + o1;
+                        }
+                    }
                 }
             }
         };
@@ -509,13 +524,49 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         acc[hw][2] += w23.x;
                         acc[hw][3] += w23.y;
                     } else {
-                        const uint16_t* vr0 =
-                            reinterpret_cast<const uint16_t*>(st + size_t(srow0) * (C::ROW * 2) + C::RK * 2) + lane;
-                        for (int j = 0; j < nv; ++j) {
-                            const float pb = __shfl_sync(0xffffffffu, pj, j);
-                            const uint16_t* vr = vr0 + j * C::ROW;
+                        // two tokens per step: half-warp `hv` takes token j0 + hv, each lane NW
+                        // 32-bit words (bf16 pairs) of c^V, word l16 + 16 k; the odd token's half
+                        // takes the words in rotated order so that the halves hit different banks
+                        constexpr int NW = C::RV / 32;
+                        const int hv = lane >> 4, l16 = lane & 15;
+                        const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + size_t(srow0 + hv) * (C::ROW * 2) +
+                                                                               C::RK * 2) + l16;
+                        uint64_t va[NW];
 #pragma unroll
-                            for (int v = 0; v < C::VPL; ++v) acc[hw][v] = fmaf(pb, bf16_to_f32(vr[32 * v]), acc[hw][v]);
+                        for (int k = 0; k < NW; ++k) va[k] = 0;
+                        if (nv == 32) {
+#pragma unroll
+                            for (int j0 = 0; j0 < 32; j0 += 2) {
+                                const float pb = __shfl_sync(0xffffffffu, pj, j0 + hv);
+                                const uint64_t pp = f2_pack(pb, pb);
+                                const uint32_t* vr = vw + j0 * (C::ROW / 2);
+#pragma unroll
+                                for (int k = 0; k < NW; ++k) {
+                                    const int kr = hv ? (k + 1 == NW ? 0 : k + 1) : k;
+                                    va[k] = f2_fma(pp, bf16x2_to_f2(vr[16 * kr]), va[k]);
+                                }
+                            }
+                        } else {
+                            // rows past the context may hold any bits: skipped, not weighted by 0
+#pragma unroll
+                            for (int j0 = 0; j0 < 32; j0 += 2) {
+                                const float pb = __shfl_sync(0xffffffffu, pj, j0 + hv);
+                                if (j0 + hv < nv) {
+                                    const uint64_t pp = f2_pack(pb, pb);
+                                    const uint32_t* vr = vw + j0 * (C::ROW / 2);
+#pragma unroll
+                                    for (int k = 0; k < NW; ++k) {
+                                        const int kr = hv ? (k + 1 == NW ? 0 : k + 1) : k;
+                                        va[k] = f2_fma(pp, bf16x2_to_f2(vr[16 * kr]), va[k]);
+                                    }
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < NW; ++k) {
+                            const float2 w = f2_unpack(va[k]);
+                            acc[hw][2 * k] += w.x;
+                            acc[hw][2 * k + 1] += w.y;
                         }
                     }
                     __syncwarp();
