@@ -83,15 +83,21 @@ struct HeadGroups {
 // make a 32-token stage of one head 16 KB: such codecs keep one head group resident (a
 // deeper stage ring) and give each lane quarter one compute warp, which walks the heads of
 // the item in turn, so that at most four stages are being read while the rest prefetch.
-template <int DH_, int RK_, int RV_, int H_, bool WIDE = (RK_ + RV_) * 2 >= 512>
-struct Cfg : HeadGroups<DH_, RK_, RV_, H_, WIDE ? 1 : 8> {
-    using HG_ = HeadGroups<DH_, RK_, RV_, H_, WIDE ? 1 : 8>;
+template <int DH_, int RK_, int RV_, int H_, bool WIDE_ = (RK_ + RV_) * 2 >= 512>
+struct Cfg : HeadGroups<DH_, RK_, RV_, H_, WIDE_ ? 1 : 8> {
+    using HG_ = HeadGroups<DH_, RK_, RV_, H_, WIDE_ ? 1 : 8>;
     using HG_::DH, HG_::RK, HG_::RV, HG_::H, HG_::HG, HG_::NG, HG_::HC, HG_::MQ_BYTES, HG_::PHI_BYTES;
     static constexpr bool TWO_D = false;
+    static constexpr bool WIDE = WIDE_;
     static constexpr int ROW = RK + RV;
     static constexpr int TOKS = (ROW * 2 * 128 <= 16384) ? 128 : (ROW * 2 * 64 <= 16384) ? 64 : 32;
     static constexpr int CHUNKS = kTile / TOKS;
     static constexpr int STAGE_BYTES = TOKS * ROW * 2;
+    // wide rows land in three panels per stage: c^K elements [0, 64) in the 128-byte swizzle,
+    // [64, r_k) in the 64-byte swizzle (bank-conflict-free row reads) and c^V as plain rows
+    static constexpr int K0_BYTES = WIDE ? TOKS * 128 : 0;
+    static constexpr int K1_BYTES = WIDE ? TOKS * (RK - 64) * 2 : 0;
+    static constexpr int V_OFF = K0_BYTES + K1_BYTES;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int FIXED = 1024 /*align slack*/ + PHI_BYTES + MQ_BYTES + BAR_BYTES;
     static constexpr int NST_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
@@ -114,12 +120,23 @@ struct Cfg : HeadGroups<DH_, RK_, RV_, H_, WIDE ? 1 : 8> {
     static constexpr int VAL = VQUAD ? RV / 4 : 32;          // lanes along the latent dimension
     static constexpr int VTL = 32 / VAL;                      // token sub-lanes
     static constexpr int VPL = VQUAD ? 4 : RV / 16;           // accumulators per lane per head
+    // two-token V path (r_v a multiple of 32 outside VQUAD): c^V row pitch in 32-bit words; a
+    // pitch that is a multiple of 32 words puts both tokens of a step on the same banks, so
+    // the odd token's half-warp takes its words in rotated order
+    static constexpr int VPW = WIDE ? RV / 2 : ROW / 2;
+    static constexpr bool VROT = VPW % 32 == 0;
     static_assert(RK % 16 == 0 && RV % 32 == 0, "ranks");
     static_assert(HC % WPQ == 0, "head split");
     static_assert(NG <= BUF_COLS, "TMEM buffer");
     static_assert(NST >= 2, "stages");
     static_assert(SMEM <= kSmemLimit, "shared memory");
     static_assert((ROW * 2) % 16 == 0, "TMA row stride");
+    static_assert(!WIDE || (RK == 96 && TOKS == 32), "wide rows: c^K split as 64 + 32 elements");
+};
+
+// Tensor maps over the layer's latents (the per-head wide layout uses all three).
+struct LatMaps {
+    CUtensorMap m[3];
 };
 
 struct TcParams {
@@ -201,8 +218,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
+__global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_constant__ LatMaps maps,
                                                                 TcParams p) {
+    const CUtensorMap& lat_map = maps.m[0];
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* phi_s = smem;
@@ -285,8 +303,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
                             break;
                         mbar_expect_tx(st_full + slot, C::STAGE_BYTES);
-                        tma_load_4d(stage_s + size_t(slot) * C::STAGE_BYTES, &lat_map, 0, h,
-                                    wk.t * kTile + ch * C::TOKS, wk.b, st_full + slot, pol_stream);
+                        uint8_t* dst = stage_s + size_t(slot) * C::STAGE_BYTES;
+                        const int tok = wk.t * kTile + ch * C::TOKS;
+                        if constexpr (C::WIDE) {
+                            tma_load_4d(dst, &maps.m[0], 0, h, tok, wk.b, st_full + slot, pol_stream);
+                            tma_load_4d(dst + C::K0_BYTES, &maps.m[1], 64, h, tok, wk.b, st_full + slot, pol_stream);
+                            tma_load_4d(dst + C::V_OFF, &maps.m[2], C::RK, h, tok, wk.b, st_full + slot, pol_stream);
+                        } else {
+                            tma_load_4d(dst, &lat_map, 0, h, tok, wk.b, st_full + slot, pol_stream);
+                        }
                         __threadfence_block();  // the armed barrier phase precedes the published round
                         issued[slot] = round + 1;
                         ++stage_k;
@@ -403,11 +428,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         for (int v = 0; v < 4; ++v) rec[2 + 4 * lane + v] = a[v];
                 } else {
                     // lane l16 < 16 holds words l16 + 16 k (k < NW) of the even tokens; lane l16 + 16
-                    // holds the odd tokens' words in rotated order: its slot k - 1 is word l16 + 16 k
+                    // holds the odd tokens' (in rotated order: its slot k - 1 is word l16 + 16 k)
                     constexpr int NW = C::RV / 32;
 #pragma unroll
                     for (int k = 0; k < NW; ++k) {
-                        const int ko = k == 0 ? NW - 1 : k - 1;
+                        const int ko = C::VROT ? (k == 0 ? NW - 1 : k - 1) : k;
                         const float o0 = __shfl_down_sync(0xffffffffu, acc[hw][2 * ko], 16);
                         const float o1 = __shfl_down_sync(0xffffffffu, acc[hw][2 * ko + 1], 16);
                         if (lane < 16) {
@@ -456,6 +481,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                     wait_stage(slot, sk / C::NST);
                     const uint8_t* st = stage_s + size_t(slot) * C::STAGE_BYTES;
                     const uint8_t* myrow = st + size_t(srow0 + lane) * (C::ROW * 2);
+                    // 16-byte chunk cc of this row's c^K (wide rows: swizzled panels)
+                    auto kchunk = [&](int cc) -> uint4 {
+                        if constexpr (C::WIDE) {
+                            if (cc < 8)
+                                return *reinterpret_cast<const uint4*>(st + lane * 128 + ((cc << 4) ^ ((lane & 7) << 4)));
+                            return *reinterpret_cast<const uint4*>(st + C::K0_BYTES + lane * 64 +
+                                                                   (((cc - 8) << 4) ^ (((lane >> 1) & 3) << 4)));
+                        } else {
+                            return *reinterpret_cast<const uint4*>(myrow + cc * 16);
+                        }
+                    };
 
                     // ---- score: s = c^K . G + bias, G read from TMEM 32 columns at a time;
                     // packed fp32 pairs: two latent dimensions per f32x2 FMA, two chains
@@ -471,7 +507,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         tmem_wait_ld();
 #pragma unroll
                         for (int c0 = 0; c0 < W; c0 += 8) {
-                            const uint4 u = *reinterpret_cast<const uint4*>(myrow + (a0 + c0) * 2);
+                            const uint4 u = kchunk((a0 + c0) >> 3);
                             s01 = f2_fma(bf16x2_to_f2(u.x), f2_pack(gv[c0 + 0], gv[c0 + 1]), s01);
                             s23 = f2_fma(bf16x2_to_f2(u.y), f2_pack(gv[c0 + 2], gv[c0 + 3]), s23);
                             s01 = f2_fma(bf16x2_to_f2(u.z), f2_pack(gv[c0 + 4], gv[c0 + 5]), s01);
@@ -525,12 +561,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         acc[hw][3] += w23.y;
                     } else {
                         // two tokens per step: half-warp `hv` takes token j0 + hv, each lane NW
-                        // 32-bit words (bf16 pairs) of c^V, word l16 + 16 k; the odd token's half
-                        // takes the words in rotated order so that the halves hit different banks
+                        // 32-bit words (bf16 pairs) of c^V, word l16 + 16 k (rotated for the odd
+                        // token when both rows of a step would meet on the same banks)
                         constexpr int NW = C::RV / 32;
                         const int hv = lane >> 4, l16 = lane & 15;
-                        const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + size_t(srow0 + hv) * (C::ROW * 2) +
-                                                                               C::RK * 2) + l16;
+                        const uint8_t* vbase = C::WIDE ? st + C::V_OFF : st + C::RK * 2;
+                        const uint32_t* vw =
+                            reinterpret_cast<const uint32_t*>(vbase + size_t(srow0 + hv) * (C::VPW * 4)) + l16;
                         uint64_t va[NW];
 #pragma unroll
                         for (int k = 0; k < NW; ++k) va[k] = 0;
@@ -539,10 +576,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                             for (int j0 = 0; j0 < 32; j0 += 2) {
                                 const float pb = __shfl_sync(0xffffffffu, pj, j0 + hv);
                                 const uint64_t pp = f2_pack(pb, pb);
-                                const uint32_t* vr = vw + j0 * (C::ROW / 2);
+                                const uint32_t* vr = vw + j0 * C::VPW;
 #pragma unroll
                                 for (int k = 0; k < NW; ++k) {
-                                    const int kr = hv ? (k + 1 == NW ? 0 : k + 1) : k;
+                                    const int kr = (C::VROT && hv) ? (k + 1 == NW ? 0 : k + 1) : k;
                                     va[k] = f2_fma(pp, bf16x2_to_f2(vr[16 * kr]), va[k]);
                                 }
                             }
@@ -553,10 +590,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                                 const float pb = __shfl_sync(0xffffffffu, pj, j0 + hv);
                                 if (j0 + hv < nv) {
                                     const uint64_t pp = f2_pack(pb, pb);
-                                    const uint32_t* vr = vw + j0 * (C::ROW / 2);
+                                    const uint32_t* vr = vw + j0 * C::VPW;
 #pragma unroll
                                     for (int k = 0; k < NW; ++k) {
-                                        const int kr = hv ? (k + 1 == NW ? 0 : k + 1) : k;
+                                        const int kr = (C::VROT && hv) ? (k + 1 == NW ? 0 : k + 1) : k;
                                         va[k] = f2_fma(pp, bf16x2_to_f2(vr[16 * kr]), va[k]);
                                     }
                                 }
@@ -849,29 +886,30 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     // 32 tokens in the 128-byte swizzle that the tensor-core operands use.
     const int h_map = C::TWO_D ? 1 : C::H;
     const size_t row_bytes = size_t(h_map) * C::ROW * 2;  // one token of one layer
-    CUtensorMap map;
+    LatMaps maps;
+    memset(&maps, 0, sizeof(maps));
     const void* base = call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
     cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(h_map), cuuint64_t(call.max_tokens), cuuint64_t(B)};
     cuuint64_t strides[3] = {cuuint64_t(C::ROW * 2), cuuint64_t(row_bytes),
                              cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
-    cuuint32_t box[4];
-    CUtensorMapSwizzle swz;
-    if constexpr (C::TWO_D) {
-        box[0] = 64u;
-        box[2] = cuuint32_t(C::QTOK);
-        swz = CU_TENSOR_MAP_SWIZZLE_128B;
-    } else {
-        box[0] = cuuint32_t(C::ROW);
-        box[2] = cuuint32_t(C::TOKS);
-        swz = CU_TENSOR_MAP_SWIZZLE_NONE;
-    }
-    box[1] = 1u;
-    box[3] = 1u;
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return LLA_ERR_CUDA;
+    auto encode = [&](CUtensorMap* m, uint32_t box_elems, uint32_t box_toks, CUtensorMapSwizzle swz) {
+        cuuint32_t box[4] = {box_elems, 1u, box_toks, 1u};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    bool enc_ok;
+    if constexpr (C::TWO_D) {
+        enc_ok = encode(&maps.m[0], 64u, C::QTOK, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else if constexpr (C::WIDE) {
+        enc_ok = encode(&maps.m[0], 64u, C::TOKS, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                 encode(&maps.m[1], C::RK - 64, C::TOKS, CU_TENSOR_MAP_SWIZZLE_64B) &&
+                 encode(&maps.m[2], C::RV, C::TOKS, CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        enc_ok = encode(&maps.m[0], C::ROW, C::TOKS, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (!enc_ok) return LLA_ERR_CUDA;
 
     TcParams tp;
     tp.phi_tiles = c->phi_tiles;
@@ -883,12 +921,12 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tp.status = pp.status;
     tp.B = B;
     tp.G = G;
-    void (*kernel)(const CUtensorMap, TcParams);
+    void (*kernel)(const LatMaps, TcParams);
     if constexpr (C::TWO_D) kernel = tc2d_decode_kernel<C>;
     else kernel = tc_decode_kernel<C>;
     LLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     if (call.ev_begin) LLA_CUDA_TRY(cudaEventRecord(call.ev_begin, call.stream));
-    kernel<<<G, C::THREADS, C::SMEM, call.stream>>>(map, tp);
+    kernel<<<G, C::THREADS, C::SMEM, call.stream>>>(maps, tp);
     LLA_CUDA_TRY(cudaGetLastError());
     if (call.ev_end) LLA_CUDA_TRY(cudaEventRecord(call.ev_end, call.stream));
     lla_tc_ranges ranges;

@@ -31,6 +31,7 @@ struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
     using HB::DH, HB::RK, HB::RV, HB::H, HB::HG, HB::NG, HB::HC, HB::GPC, HB::MQ_BYTES, HB::MQ_GROUP_BYTES,
         HB::PHI_BYTES;
     static constexpr bool TWO_D = true;
+    static constexpr bool WIDE = false;
     static constexpr int ROW = RK + RV;
     static constexpr int QTOK = 32;                     // tokens per TMEM lane quarter
     static constexpr int PANEL = QTOK * 128;            // one 64-wide swizzled panel of a quarter
@@ -74,8 +75,9 @@ __device__ __forceinline__ void wait_last_phases(uint64_t* bars, uint32_t ns, ui
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid_constant__ CUtensorMap lat_map,
+__global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid_constant__ LatMaps maps,
                                                                   TcParams p) {
+    const CUtensorMap& lat_map = maps.m[0];
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* phi_s = smem;                               // [NPHI][PHI_BYTES]
