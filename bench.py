@@ -41,7 +41,7 @@ DEFAULT_WORKLOAD = "ouro_rho21_b768_n4096"
 # kernels the library launches per call (our own kernels only; memsets excluded)
 LAUNCHES_PER_DECODE = {"simt": 2, "tc": 3}
 LAUNCHES_PER_ENCODE = 1
-KERNEL_SOURCES = {"simt": "decode_simt.cu", "tc": "decode_tc.cu"}
+KERNEL_SOURCES = {"simt": ["decode_simt.cu", "sm100.cuh"], "tc": ["decode_tc.cu", "decode_tc2d.cuh", "sm100.cuh"]}
 
 
 def parse():
@@ -217,26 +217,66 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------------------------
 
-def measured_peak():
+def measured_peak(key="hbm_gbs"):
+    """(peak, "measured"|"fallback"): HBM GB/s, or dense bf16 TFLOP/s ("bf16_tflops_sustained")."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
-        return float(j["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        if key in j:
+            return float(j[key]), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}[key], "fallback"
 
 
-def traffic_record(kernel):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
-    src = os.path.join(ROOT, "decode_attention_lla_b200", "csrc", KERNEL_SOURCES[kernel])
-    rec = os.path.join(ROOT, "profiles", f"traffic_{kernel}.json")
-    if not (os.path.exists(src) and os.path.exists(rec)):
+def flops_per_call(cfg):
+    """Algorithmic tensor-core work of one decode call: reconstructing every head's keys from the
+    latents, [tokens x r_k] . [r_k x H d] (the position-GEMM form does the same contraction)."""
+    return 2.0 * cfg["batch"] * cfg["context"] * cfg["H"] * cfg["d_head"] * cfg["r_k"]
+
+
+def roofline(cfg, kernel_name, kern_ms, workload):
+    """The bound that binds the decode kernel: HBM for per-head latents, tensor cores for LLA-2D
+    on the tensor-core kernel (683 flop per latent byte).  The kernel is timed inside a long
+    step, so the tensor peak is the sustained figure."""
+    kmean = statistics.mean(kern_ms)
+    byt = bytes_per_call(cfg)
+    hbm_peak, hbm_kind = measured_peak("hbm_gbs")
+    hbm_achieved = byt / (kmean / 1e3) / 1e9
+    r = {"kernel": f"lla decode ({kernel_name})", "kernel_ms_mean": kmean, "kernel_ms_min": min(kern_ms),
+         "algorithmic_bytes_per_launch": byt}
+    if cfg["variant"] == 1 and kernel_name == "tc":
+        tf_peak, tf_kind = measured_peak("bf16_tflops_sustained")
+        fl = flops_per_call(cfg)
+        achieved = fl / (kmean / 1e3) / 1e12
+        r.update({"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                  "frac": achieved / tf_peak, "traffic": traffic_record(kernel_name, workload),
+                  "peak_source": f"{tf_kind} bf16_tflops_sustained (fp16 operands: same dense rate)",
+                  "algorithmic_flops_per_launch": fl, "hbm_achieved_gbs": hbm_achieved,
+                  "hbm_frac": hbm_achieved / hbm_peak})
+    else:
+        r.update({"bound": "hbm", "achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                  "frac": hbm_achieved / hbm_peak, "traffic": traffic_record(kernel_name, workload),
+                  "peak_source": f"{hbm_kind} hbm_gbs"})
+    return r
+
+
+def kernel_sha(kernel):
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "decode_attention_lla_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_record(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary of this kernel on this workload, if it
+    was taken on the current kernel sources (else None)."""
+    rec = os.path.join(ROOT, "profiles", f"traffic_{kernel}_{workload}.json")
+    if not os.path.exists(rec):
         return None
-    with open(src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()
     with open(rec) as f:
         j = json.load(f)
-    return j.get("dram_bytes_per_launch") if j.get("source_sha256") == h else None
+    return j.get("dram_bytes_per_launch") if j.get("source_sha256") == kernel_sha(kernel) else None
 
 
 def run_ours(a, cfg):
@@ -365,19 +405,12 @@ def run_ours(a, cfg):
     d2h = T * D * B * H * d * 4
 
     if rank == 0:
-        peak, peak_kind = measured_peak()
-        kmean = statistics.mean(kern_ms)
-        achieved = bytes_per_call(cfg) / (kmean / 1e3) / 1e9
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": config_json(cfg, a.workload, world),
                 "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
-                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": traffic_record(kernel_name),
-                             "kernel": f"lla decode ({kernel_name})", "peak_source": f"{peak_kind} hbm_gbs",
-                             "kernel_ms_mean": kmean, "kernel_ms_min": min(kern_ms),
-                             "algorithmic_bytes_per_launch": bytes_per_call(cfg)},
+                "roofline": roofline(cfg, kernel_name, kern_ms, a.workload),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "clocks": clk.summary(),
                 "gpu_launches": a.steps * (T * D * LAUNCHES_PER_DECODE[kernel_name] + LAUNCHES_PER_ENCODE)}

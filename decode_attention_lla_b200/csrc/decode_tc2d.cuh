@@ -153,7 +153,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         // ------------------------------------------------------------ M_q, Phi, c^K loads
         if (elect_one()) {
             prefetch_tensormap(&lat_map);
-            const uint64_t pol_stream = policy_evict_first();
+            // a latent tile is read by every head part of the group within a short time: plain
+            // L2 priority keeps it for them (evict-first let it go before the last part's read)
+            const uint64_t pol_stream = policy_evict_normal();
             const uint64_t pol_keep = policy_evict_last();
             uint32_t kk_n = 0, phi_n = 0, mq_n = 0;
             int prev_key = -1;
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     } else if (warp == 2) {
         // ------------------------------------------------------------ c^V loads
         if (elect_one()) {
-            const uint64_t pol_stream = policy_evict_first();
+            const uint64_t pol_stream = policy_evict_normal();
             uint32_t vk_n = 0;
             bool ok = true;
             for (; wk.valid() && ok; wk.next()) {

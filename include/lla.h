@@ -162,7 +162,9 @@ lla_status lla_decode_attn(const lla_codec* codec, const uint16_t* store, int ba
  * lla_decode_attn_2d — LLA-2D decode attention [LLA §3, "LLA-2D variant"].
  *   Same arguments as lla_decode_attn; the codec must have variant 1 and the
  *   store is [batch][D][max_tokens][r_k + r_v]: one latent per token decodes
- *   all H heads through per-(loop, head) up-projections.
+ *   all H heads through per-(loop, head) up-projections.  On the tcgen05
+ *   kernel the latent-space V sum is a tensor-core GEMM whose attention
+ *   weights are bf16 (the softmax denominator sums the same rounded weights).
  */
 lla_status lla_decode_attn_2d(const lla_codec* codec, const uint16_t* store, int batch,
                               int max_tokens, int layer, int loop, const float* q,
