@@ -105,8 +105,12 @@ def attention(q, Ks, Vs, scale):
     return [sum(w[j] * Vs[j][i] for j in range(len(Vs))) / z for i in range(dv)]
 
 
-def decode_head(q, cK, cV, muKt, WKt, muVt, WVt, pos_q, scale, base):
-    """Loop-t attention of one head over its cached latents (token j at position j)."""
+def decode_head(q, cK, cV, muKt, WKt, muVt, WVt, pos_q, scale, base, k_self=None, v_self=None):
+    """Loop-t attention of one head over its cached latents (token j at position j), plus the
+    current token's exact key and value as one more slot at the query's position when given."""
     Ks = [rope(reconstruct(c, WKt, muKt), j, base) for j, c in enumerate(cK)]
     Vs = [reconstruct(c, WVt, muVt) for c in cV]
+    if k_self is not None:
+        Ks.append(rope(list(k_self), pos_q, base))
+        Vs.append(list(v_self))
     return attention(rope(q, pos_q, base), Ks, Vs, scale)

@@ -25,6 +25,10 @@ Readings of points the paper leaves open (each also listed in the design doc):
 * mu_t is the loop-t slice of mu; W_up,t is independent of W_down (they
   coincide only at SVD initialisation).
 * An empty context (seq_len == 0) yields a zero output.
+* Self slot (optional): the current token's latent is written only after
+  its last loop, so at decode time its own loop-t key and value are the
+  loop's exact vectors; when given, they join the attention as one more
+  slot at the query's position.
 
 Parity pins: every public function here is checked by ``tests/test_oracle_*``
 against closed forms, printed numbers, special cases that reduce to library
@@ -203,7 +207,7 @@ def softmax_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float)
     return (w / w.sum()) @ V
 
 
-def lla_decode_head(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base):
+def lla_decode_head(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base, k_self=None, v_self=None):
     """Loop-t decode attention for one (sequence, head) from latents.
 
     cK [n, r_k], cV [n, r_v] are the cached latents of tokens 0..n-1 (token j
@@ -211,6 +215,11 @@ def lla_decode_head(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base)
     applied to the reconstructed keys and to the query, and softmax attention
     follows [LLA §3 eq. (3); "RoPE and reconstruction"].  The latent-space
     shortcut for V is deliberately NOT used here.
+
+    k_self, v_self [d] (optional): the current token's exact loop-t key
+    (pre-RoPE) and value.  Its latent does not exist yet (eq. (2) needs the
+    whole loop stack), so it joins as one more slot, key rotated at the
+    query's position.
     """
     cK = np.asarray(cK, np.float64)
     n = cK.shape[0]
@@ -218,10 +227,13 @@ def lla_decode_head(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base)
     V_hat = reconstruct(cV, WupV_t, muV_t)
     K_rot = apply_rope(K_hat, np.arange(n), base)
     q_rot = apply_rope(q, pos_q, base)
+    if k_self is not None:
+        K_rot = np.vstack([K_rot, apply_rope(k_self, pos_q, base)[None]])
+        V_hat = np.vstack([V_hat, np.asarray(v_self, np.float64)[None]])
     return softmax_attention(q_rot, K_rot, V_hat, scale)
 
 
-def lla_decode(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, base):
+def lla_decode(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, base, k_self=None, v_self=None):
     """Per-head LLA decode attention for one (layer, loop) call.
 
     q       [B, H, d]          pre-RoPE queries
@@ -231,6 +243,7 @@ def lla_decode(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, ba
     WupK    [H, T, d, r_k]     W_up,t of the K codec        (WupV alike)
     loop    t in [0, T)
     seq_lens[B], q_pos[B]      context length and query position per sequence
+    k_self, v_self [B, H, d]   optional self slot (see lla_decode_head)
     Returns out [B, H, d].
     """
     q = np.asarray(q, np.float64)
@@ -239,9 +252,11 @@ def lla_decode(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, ba
     for b in range(B):
         n = int(seq_lens[b])
         for h in range(H):
+            ks = None if k_self is None else k_self[b, h]
+            vs = None if v_self is None else v_self[b, h]
             out[b, h] = lla_decode_head(q[b, h], cK[b, :n, h], cV[b, :n, h],
                                         muK[h, loop], WupK[h, loop], muV[h, loop], WupV[h, loop],
-                                        float(q_pos[b]), scale, base)
+                                        float(q_pos[b]), scale, base, ks, vs)
     return out
 
 
@@ -258,14 +273,15 @@ def encode_2d(x, mu, W_down):
     return encode(x, mu, W_down)
 
 
-def lla_decode_2d(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, base):
+def lla_decode_2d(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale, base, k_self=None, v_self=None):
     """LLA-2D decode attention: one latent per token decodes all H heads.
 
     q    [B, H, d]
     cK   [B, N, r_k], cV [B, N, r_v]   one latent per token (per layer)
     muK  [T, H, d], WupK [T, H, d, r_k] per-(loop, head) slices (V alike)
     Head h at loop t reconstructs x_hat_{t,h} = c W_up,(t,h)^T + mu_{t,h}
-    [LLA §3, "LLA-2D variant"]; RoPE and attention as in the per-head case.
+    [LLA §3, "LLA-2D variant"]; RoPE, attention and the optional self slot
+    (k_self, v_self [B, H, d]) as in the per-head case.
     """
     q = np.asarray(q, np.float64)
     B, H, d = q.shape
@@ -273,7 +289,9 @@ def lla_decode_2d(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale,
     for b in range(B):
         n = int(seq_lens[b])
         for h in range(H):
+            ks = None if k_self is None else k_self[b, h]
+            vs = None if v_self is None else v_self[b, h]
             out[b, h] = lla_decode_head(q[b, h], cK[b, :n], cV[b, :n],
                                         muK[loop, h], WupK[loop, h], muV[loop, h], WupV[loop, h],
-                                        float(q_pos[b]), scale, base)
+                                        float(q_pos[b]), scale, base, ks, vs)
     return out

@@ -25,6 +25,8 @@ PIN_TESTS = [
     pins.test_single_loop_full_rank_is_textbook_rope_attention,
     pins.test_v_identity_in_latent_space,
     pins.test_softmax_special_cases,
+    pins.test_self_slot_with_empty_cache_is_its_value,
+    pins.test_self_slot_matches_sdpa_over_the_appended_token,
     lambda: pins.test_vectorised_oracle_matches_brute_force(dict(T=2, d=4, rk=2, rv=3, n=8, H=2, B=2)),
 ]
 
@@ -80,18 +82,41 @@ def _fit_uncentred(X, r):
     return mu, vt[:r].T.copy(), s2
 
 
-def _decode_shift_positions(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base):
+def _with_self(K, V, k_self, v_self, pos_q, base, self_pos=None):
+    if k_self is None:
+        return K, V
+    p = pos_q if self_pos is None else self_pos
+    return (np.vstack([K, O.apply_rope(k_self, p, base)[None]]),
+            np.vstack([V, np.asarray(v_self, np.float64)[None]]))
+
+
+def _decode_shift_positions(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base, k_self=None, v_self=None):
     n = np.asarray(cK).shape[0]
     K = O.apply_rope(O.reconstruct(cK, WupK_t, muK_t), np.arange(1, n + 1), base)
     V = O.reconstruct(cV, WupV_t, muV_t)
+    K, V = _with_self(K, V, k_self, v_self, pos_q, base)
     return O.softmax_attention(O.apply_rope(q, pos_q, base), K, V, scale)
 
 
-def _decode_rope_on_v(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base):
+def _decode_rope_on_v(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base, k_self=None, v_self=None):
     n = np.asarray(cK).shape[0]
     K = O.apply_rope(O.reconstruct(cK, WupK_t, muK_t), np.arange(n), base)
     V = O.apply_rope(O.reconstruct(cV, WupV_t, muV_t), np.arange(n), base)
+    K, V = _with_self(K, V, k_self, v_self, pos_q, base)
     return O.softmax_attention(O.apply_rope(q, pos_q, base), K, V, scale)
+
+
+def _decode_self_unrotated(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base, k_self=None, v_self=None):
+    """The self key enters at position 0 instead of the query's position."""
+    n = np.asarray(cK).shape[0]
+    K = O.apply_rope(O.reconstruct(cK, WupK_t, muK_t), np.arange(n), base)
+    V = O.reconstruct(cV, WupV_t, muV_t)
+    K, V = _with_self(K, V, k_self, v_self, pos_q, base, self_pos=0.0)
+    return O.softmax_attention(O.apply_rope(q, pos_q, base), K, V, scale)
+
+
+def _decode_self_dropped(q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base, k_self=None, v_self=None):
+    return _orig["lla_decode_head"](q, cK, cV, muK_t, WupK_t, muV_t, WupV_t, pos_q, scale, base)
 
 
 def _store_bytes_fp32(batch, tokens, D, H, r_k, r_v, variant=0, bytes_per_scalar=2):
@@ -114,6 +139,8 @@ MUTATIONS = {
     "SVD fit on uncentred stacks": ("fit_codec_svd", _fit_uncentred),
     "keys at positions 1..n": ("lla_decode_head", _decode_shift_positions),
     "RoPE applied to values": ("lla_decode_head", _decode_rope_on_v),
+    "self key not rotated to the query position": ("lla_decode_head", _decode_self_unrotated),
+    "self slot dropped": ("lla_decode_head", _decode_self_dropped),
     "store counted in fp32": ("store_bytes", _store_bytes_fp32),
     "teacher cache counts one axis": ("uncompressed_scalars_per_token_layer", _scalars_one_axis),
 }

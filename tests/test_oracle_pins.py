@@ -241,6 +241,36 @@ def test_v_identity_in_latent_space():
     assert np.abs(got - ((p @ cV) @ WV.T + muV)).max() < 1e-13
 
 
+def test_self_slot_with_empty_cache_is_its_value():
+    """With no cached token the softmax has the self slot alone: the output is v_self."""
+    d, rk, rv = 8, 3, 5
+    q = syn.gaussian("pin/self0/q", d)
+    ks, vs = syn.gaussian("pin/self0/k", d), syn.gaussian("pin/self0/v", d)
+    W = syn.gaussian("pin/self0/W", (d, rk))
+    got = O.lla_decode_head(q, np.zeros((0, rk)), np.zeros((0, rv)), np.zeros(d), W, np.zeros(d),
+                            np.zeros((d, rv)), 11.0, 0.5, 10000.0, ks, vs)
+    assert np.abs(got - vs).max() < 1e-15
+
+
+def test_self_slot_matches_sdpa_over_the_appended_token():
+    """Self slot = one more key/value row, the key rotated at the query's position."""
+    d, rk, rv, n, pos = 16, 4, 6, 25, 31.0
+    cK, cV = syn.gaussian("pin/self/cK", (n, rk)), syn.gaussian("pin/self/cV", (n, rv))
+    WK, WV = syn.gaussian("pin/self/WK", (d, rk), 0.3), syn.gaussian("pin/self/WV", (d, rv), 0.3)
+    muK, muV = syn.gaussian("pin/self/muK", d), syn.gaussian("pin/self/muV", d)
+    q = syn.gaussian("pin/self/q", d)
+    ks, vs = syn.gaussian("pin/self/k", d), syn.gaussian("pin/self/v", d)
+    got = O.lla_decode_head(q, cK, cV, muK, WK, muV, WV, pos, 0.3, 10000.0, ks, vs)
+    K = np.vstack([rope_complex(cK @ WK.T + muK, np.arange(n), 10000.0), rope_complex(ks, pos, 10000.0)[None]])
+    V = np.vstack([cV @ WV.T + muV, vs[None]])
+    ref = sdpa(rope_complex(q, pos, 10000.0), K, V, 0.3)
+    assert np.abs(got - ref).max() < 1e-12
+    # query and self key share one rotation, which cancels: the self logit is scale * <q, k_self>
+    lg = np.append(0.3 * K[:n] @ rope_complex(q, pos, 10000.0), 0.3 * q @ ks)
+    p = np.exp(lg - lg.max())
+    assert np.abs(got - (p / p.sum()) @ V).max() < 1e-12
+
+
 def test_softmax_special_cases():
     d, n = 8, 12
     V = syn.gaussian("pin/sm/V", (n, d))
@@ -297,14 +327,19 @@ def test_vectorised_oracle_matches_brute_force(case):
     muV = np.stack([mVt] * H)
     WupK = np.stack([WKt] * H)
     WupV = np.stack([WVt] * H)
+    ks, vs = syn.gaussian(tag + "/ks", (B, H, d)), syn.gaussian(tag + "/vs", (B, H, d))
     for t in range(T):
         got = O.lla_decode(q, cK, cV, muK, WupK, muV, WupV, t, lens, qpos, scale, base)
+        got_self = O.lla_decode(q, cK, cV, muK, WupK, muV, WupV, t, lens, qpos, scale, base, ks, vs)
         for b in range(B):
             for h in range(H):
-                ref = bf.decode_head(q[b, h].tolist(), cK[b, :lens[b], h].tolist(), cV[b, :lens[b], h].tolist(),
-                                     mKt[t].tolist(), WKt[t].tolist(), mVt[t].tolist(), WVt[t].tolist(),
-                                     float(qpos[b]), scale, base)
+                args = (q[b, h].tolist(), cK[b, :lens[b], h].tolist(), cV[b, :lens[b], h].tolist(),
+                        mKt[t].tolist(), WKt[t].tolist(), mVt[t].tolist(), WVt[t].tolist(), float(qpos[b]), scale,
+                        base)
+                ref = bf.decode_head(*args)
                 assert np.abs(got[b, h] - np.array(ref)).max() < 1e-12
+                ref_self = bf.decode_head(*args, ks[b, h].tolist(), vs[b, h].tolist())
+                assert np.abs(got_self[b, h] - np.array(ref_self)).max() < 1e-12
 
 
 def test_tiny_workload_codec_properties():
