@@ -70,10 +70,13 @@ _decode_2d = _sig("lla_decode_attn_2d", _i, _decode_args + [_vp])
 _decode_ex = _sig("lla_decode_attn_ex", _i, _decode_args + [ctypes.POINTER(DecodeOpts), _vp])
 _flags = _sig("lla_workspace_flags", _i, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp])
 _decode_noalloc = _sig("lla_decode_attn_noalloc", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp])
+_decode_self = _sig("lla_decode_attn_self", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _sz,
+                                                 ctypes.POINTER(DecodeOpts), _vp])
 
 EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy_codec", "lla_codec_get_desc",
             "lla_store_bytes", "lla_encode", "lla_decode_workspace_bytes", "lla_decode_attn",
-            "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc"]
+            "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc",
+            "lla_decode_attn_self"]
 
 
 class LLAError(RuntimeError):
@@ -228,9 +231,23 @@ def decode_attn_2d(codec, store, batch, max_tokens, layer, loop, q, q_pos, seq_l
                         workspace, workspace_bytes, stream), "lla_decode_attn_2d")
 
 
+def decode_attn_self(codec, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, k_self, v_self, scale, out,
+                     workspace, workspace_bytes=None, stream=None, impl=IMPL_AUTO, num_ctas=0, events=None):
+    """lla_decode_attn_self: decode attention with the current token's exact loop-t key and value
+    (k_self, v_self [batch][H][d_head] float32) as one more softmax slot; either codec variant."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    opts = DecodeOpts(impl, num_ctas, *(events if events is not None else (None, None)))
+    st = _decode_self(codec.handle, _ptr(store), batch, max_tokens, layer, loop, _ptr(q), _ptr(q_pos),
+                      _ptr(seq_lens), _ptr(k_self), _ptr(v_self), float(scale), _ptr(out), _ptr(workspace),
+                      int(workspace_bytes), ctypes.byref(opts), _stream(stream))
+    _check(st, "lla_decode_attn_self")
+
+
 def raw_decode_status(fn_name, *args) -> int:
     """Call a decode entry point with raw arguments and return its status (for ABI tests)."""
-    return {"lla_decode_attn": _decode, "lla_decode_attn_2d": _decode_2d, "lla_decode_attn_ex": _decode_ex}[fn_name](*args)
+    return {"lla_decode_attn": _decode, "lla_decode_attn_2d": _decode_2d, "lla_decode_attn_ex": _decode_ex,
+            "lla_decode_attn_self": _decode_self}[fn_name](*args)
 
 
 def workspace_flags(workspace, stream=None) -> int:

@@ -8,6 +8,12 @@
 // which equals sum_j p_j v_hat_j because the normalised p_j sum to one
 // [LLA §3 eq. (3)].  An empty context (no records with l > 0) yields zeros.
 //
+// Optional self slot: the current token's exact loop-t key and value join the softmax as one
+// more term.  Query and self key sit at the same position, so their rotations cancel and the
+// logit is scale * <q, k_self>; with w_self its normalised weight,
+//   out = (sum_s w_s acc_s) W^V_up,t^T + (1 - w_self) mu^V_t + w_self v_self,
+// since the cached tokens then carry 1 - w_self of the probability.
+//
 // One CTA per (head, 16 sequences), one warp per sequence: W^V_up,t of the head
 // is staged in shared memory once, transposed so that the lanes of a warp (one
 // output dimension each) read consecutive words.
@@ -30,6 +36,11 @@ struct CombineParams {
     // tensor-core record layout (tc_P != null): see lla_tc_ranges
     const int32_t* tc_P;
     int tc_G, tc_parts, tc_hc;
+    // self slot (k_self == null: none)
+    const float* q;
+    const float* k_self;
+    const float* v_self;
+    float scale;
 };
 
 // The records of (b, h): rec(s) for s in [0, n).
@@ -121,9 +132,19 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     const RecordSet rs = record_set(p, b, h);
     auto rec = [&](int s) { return rs.rec(s); };
     const int s0 = 0, s1 = rs.n;
+    const size_t bh = size_t(b) * p.H + h;
+    // self-slot logit (natural-log units, like the records' m)
+    float s_self = -INFINITY;
+    if (p.k_self) {
+        float dot = 0.f;
+        for (int i = lane; i < d; i += 32) dot = fmaf(p.q[bh * d + i], p.k_self[bh * d + i], dot);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        s_self = p.scale * dot;
+    }
     // merged maximum and normaliser over the records (log-sum-exp); a record with l = 0
     // saw no valid token and is skipped whatever its m holds
-    float M = -INFINITY;
+    float M = s_self;
     for (int s = s0 + lane; s < s1; s += 32) {
         const float* r = rec(s);
         if (r[1] > 0.f) M = fmaxf(M, r[0]);
@@ -138,11 +159,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
         }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    float* o = p.out + (size_t(b) * p.H + h) * d;
+    const float e_self = p.k_self ? expf(s_self - M) : 0.f;
+    L += e_self;
+    float* o = p.out + bh * d;
     if (!(L > 0.f)) {  // empty context
         for (int i = lane; i < d; i += 32) o[i] = 0.f;
         return;
     }
+    const float w_self = e_self / L;
     // record weights exp(m_s - M) / L, one per lane, broadcast by shuffle
     const float invL = 1.f / L;
     for (int a = lane; a < rv; a += 32) abar[a] = 0.f;
@@ -165,9 +189,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
         }
     }
     __syncwarp();
-    // out = abar W^V_up,t^T + mu^V_t
+    // out = abar W^V_up,t^T + (1 - w_self) mu^V_t + w_self v_self
     for (int i = lane; i < d; i += 32) {
-        float v = mu[i];
+        float v = p.k_self ? fmaf(w_self, p.v_self[bh * d + i], (1.f - w_self) * mu[i]) : mu[i];
         for (int a = 0; a < rv; ++a) v = fmaf(abar[a], Wt[a * d + i], v);
         o[i] = v;
     }
@@ -213,6 +237,10 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     p.layer = call.layer;
     p.loop = call.loop;
     p.variant = ds.variant;
+    p.q = call.q;
+    p.k_self = call.k_self;
+    p.v_self = call.v_self;
+    p.scale = call.scale;
     const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     dim3 grid(ds.H, (call.batch + kSeqPerCta - 1) / kSeqPerCta);

@@ -230,7 +230,8 @@ size_t lla_decode_workspace_bytes(const lla_codec* c, int batch, int max_tokens)
 static lla_status decode_common(int want_variant, const lla_codec* c, const uint16_t* store, int batch,
                                 int max_tokens, int layer, int loop, const float* q, const int32_t* q_pos,
                                 const int32_t* seq_lens, float scale, float* out, void* workspace,
-                                size_t workspace_bytes, const lla_decode_opts* opts, void* stream) {
+                                size_t workspace_bytes, const lla_decode_opts* opts, void* stream,
+                                const float* k_self = nullptr, const float* v_self = nullptr) {
     if (!c || c->desc.variant != want_variant) return LLA_ERR_INVALID_ARG;
     if (batch < 0 || max_tokens < 0 || layer < 0 || layer >= c->desc.D || loop < 0 || loop >= c->desc.T)
         return LLA_ERR_INVALID_ARG;
@@ -241,6 +242,8 @@ static lla_status decode_common(int want_variant, const lla_codec* c, const uint
     if (!aligned16(store) || !aligned16(q) || !aligned16(out) || !aligned16(workspace) || !aligned4(q_pos) ||
         !aligned4(seq_lens))
         return LLA_ERR_ALIGNMENT;
+    if ((k_self == nullptr) != (v_self == nullptr)) return LLA_ERR_INVALID_ARG;
+    if (k_self && (!aligned16(k_self) || !aligned16(v_self))) return LLA_ERR_ALIGNMENT;
     if (workspace_bytes < lla_decode_workspace_bytes(c, batch, max_tokens)) return LLA_ERR_WORKSPACE;
     const int impl = opts ? opts->impl : 0;
     const int num_ctas = opts ? opts->num_ctas : 0;
@@ -265,9 +268,14 @@ static lla_status decode_common(int want_variant, const lla_codec* c, const uint
         call.ev_begin = static_cast<cudaEvent_t>(opts->ev_begin);
         call.ev_end = static_cast<cudaEvent_t>(opts->ev_end);
     }
+    call.k_self = k_self;
+    call.v_self = v_self;
     LLA_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(lla_ws_header), call.stream));
     if (max_tokens == 0) {
-        LLA_CUDA_TRY(cudaMemsetAsync(out, 0, size_t(batch) * c->desc.H * c->desc.d_head * 4, call.stream));
+        // no cached token: the softmax is empty (zero output) or the self slot alone (its value)
+        const size_t bytes = size_t(batch) * c->desc.H * c->desc.d_head * 4;
+        if (v_self) LLA_CUDA_TRY(cudaMemcpyAsync(out, v_self, bytes, cudaMemcpyDeviceToDevice, call.stream));
+        else LLA_CUDA_TRY(cudaMemsetAsync(out, 0, bytes, call.stream));
         return LLA_OK;
     }
     const bool tc_ok = lla_tc_supported(c);
@@ -297,6 +305,17 @@ lla_status lla_decode_attn_ex(const lla_codec* c, const uint16_t* store, int bat
     if (!c) return LLA_ERR_INVALID_ARG;
     return decode_common(c->desc.variant, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out,
                          workspace, workspace_bytes, opts, stream);
+}
+
+lla_status lla_decode_attn_self(const lla_codec* c, const uint16_t* store, int batch, int max_tokens, int layer,
+                                int loop, const float* q, const int32_t* q_pos, const int32_t* seq_lens,
+                                const float* k_self, const float* v_self, float scale, float* out,
+                                void* workspace, size_t workspace_bytes, const lla_decode_opts* opts,
+                                void* stream) {
+    if (!c) return LLA_ERR_INVALID_ARG;
+    if (batch > 0 && (!k_self || !v_self)) return LLA_ERR_INVALID_ARG;
+    return decode_common(c->desc.variant, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out,
+                         workspace, workspace_bytes, opts, stream, k_self, v_self);
 }
 
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {

@@ -63,6 +63,8 @@ struct lla_decode_call {
     cudaStream_t stream;
     cudaEvent_t ev_begin = nullptr;  // recorded around the main attention kernel when set
     cudaEvent_t ev_end = nullptr;
+    const float* k_self = nullptr;   // optional self slot: the current token's exact loop-t
+    const float* v_self = nullptr;   // key (pre-RoPE) and value, [batch][H][d_head]
 };
 
 // ---- bf16 helpers ---------------------------------------------------------

@@ -200,6 +200,32 @@ lla_status lla_decode_attn_ex(const lla_codec* codec, const uint16_t* store, int
                               void* stream);
 
 /*
+ * lla_decode_attn_self — decode attention with the current token as a self slot
+ *   [LLA §3 eq. (2)-(3)]: a token's latent is written only after its last loop
+ *   (eq. (2) encodes the whole loop stack), so while it is being decoded its
+ *   own loop-t key and value are the loop's exact vectors.  They join the
+ *   softmax as one more slot at the query's position:
+ *     out_bh = sum over the n cached tokens and the self slot of
+ *              softmax(s)_j v_j,  s_self = softmax_scale * <q_bh, k_self_bh>
+ *   (query and self key share one rotation, which cancels in the product).
+ *   Arguments as lla_decode_attn (either codec variant: per-head or 2D store),
+ *   plus
+ *   k_self    device float32 [batch][H][d_head], the current token's loop-t
+ *             key before RoPE, 16-byte aligned
+ *   v_self    device float32 [batch][H][d_head], its loop-t value
+ *   opts      as lla_decode_attn_ex, or NULL.
+ *   With n == 0 the output is v_self.  Errors as lla_decode_attn; a NULL
+ *   k_self or v_self with batch > 0 is LLA_ERR_INVALID_ARG.
+ */
+lla_status lla_decode_attn_self(const lla_codec* codec, const uint16_t* store, int batch,
+                                int max_tokens, int layer, int loop, const float* q,
+                                const int32_t* q_pos, const int32_t* seq_lens,
+                                const float* k_self, const float* v_self,
+                                float softmax_scale, float* out, void* workspace,
+                                size_t workspace_bytes, const lla_decode_opts* opts,
+                                void* stream);
+
+/*
  * lla_workspace_flags — read the device status word of a decode workspace
  * (synchronises `stream`).  Bit 0: a seq_len was above max_tokens (clamped);
  * bit 1: a key or query position was outside [0, max_pos) (clamped).  The

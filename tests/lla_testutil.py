@@ -93,19 +93,19 @@ def unpack_layer(store_bits: np.ndarray, layer: int, rk: int):
     return s[..., :rk], s[..., rk:]
 
 
-def oracle_decode(codec: dict, cfg: dict, cK, cV, q, layer, loop, seq_lens, q_pos, scale):
-    """Oracle output for one (layer, loop) call; codec is the rounded dict."""
+def oracle_decode(codec: dict, cfg: dict, cK, cV, q, layer, loop, seq_lens, q_pos, scale, k_self=None, v_self=None):
+    """Oracle output for one (layer, loop) call; codec is the rounded dict; optional self slot."""
     T, H, d = cfg["T"], cfg["H"], cfg["d_head"]
     base = cfg.get("rope_base", 10000.0)
     if cfg["variant"] == 0:
         muK = codec["mu_k"][layer].reshape(H, T, d)
         muV = codec["mu_v"][layer].reshape(H, T, d)
         return O.lla_decode(q, cK, cV, muK, codec["w_up_k"][layer], muV, codec["w_up_v"][layer], loop,
-                            seq_lens, q_pos, scale, base)
+                            seq_lens, q_pos, scale, base, k_self, v_self)
     muK = codec["mu_k"][layer].reshape(T, H, d)
     muV = codec["mu_v"][layer].reshape(T, H, d)
     return O.lla_decode_2d(q, cK, cV, muK, codec["w_up_k"][layer], muV, codec["w_up_v"][layer], loop,
-                           seq_lens, q_pos, scale, base)
+                           seq_lens, q_pos, scale, base, k_self, v_self)
 
 
 def default_scale(d: int) -> float:
