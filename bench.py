@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--mode", choices=["decode", "encode"], default="decode",
                     help="encode: time prefill encoding of teacher stacks instead of the decode step")
     ap.add_argument("--encode-tokens", type=int, default=4096, help="tokens per encode call (encode mode)")
+    ap.add_argument("--self-slot", action="store_true",
+                    help="decode calls attend to the current token's exact K/V as well (lla_decode_attn_self)")
     return ap.parse_args()
 
 
@@ -311,6 +313,10 @@ def run_ours(a, cfg):
     q_all.normal_(generator=syn.torch_generator(tag + "/q", dev))
     S = T * d if cfg["variant"] == 0 else T * H * d
     x_shape = (B, D, H, 2, S) if cfg["variant"] == 0 else (B, D, 2, S)
+    kv_self = None
+    if a.self_slot:  # the current token's exact loop-t key and value per call: [T][D][2][B][H][d]
+        kv_self = torch.empty(T, D, 2, B, H, d, dtype=torch.float32, device=dev)
+        kv_self.normal_(generator=syn.torch_generator(tag + "/kv_self", dev))
     x_new = torch.empty(x_shape, dtype=torch.bfloat16, device=dev)
     x_new.normal_(generator=syn.torch_generator(tag + "/x", dev))
     seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
@@ -340,8 +346,16 @@ def run_ours(a, cfg):
                     q = host["q_dev"]
                     q.copy_(host["q"][t, layer], non_blocking=True)
                 ev = events[k] if events is not None else None
-                lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl,
-                                events=ev)
+                if kv_self is None:
+                    lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl,
+                                    events=ev)
+                else:
+                    kv = kv_self[t, layer]
+                    if host is not None:
+                        kv = host["kv_dev"]
+                        kv.copy_(host["kv"][t, layer], non_blocking=True)
+                    lla.decode_attn_self(codec, store, B, cap, layer, t, q, qpos, lens, kv[0], kv[1], scale, out,
+                                         ws, impl=impl, events=ev)
                 if host is not None:
                     host["out"][t, layer].copy_(out, non_blocking=True)
                 k += 1
@@ -389,6 +403,10 @@ def run_ours(a, cfg):
                 "x": torch.empty(x_shape, dtype=torch.bfloat16, pin_memory=True),
                 "q_dev": torch.empty(B, H, d, dtype=torch.float32, device=dev)}
         host["q"].copy_(q_all.cpu())
+        if kv_self is not None:
+            host["kv"] = torch.empty(kv_self.shape, dtype=torch.float32, pin_memory=True)
+            host["kv"].copy_(kv_self.cpu())
+            host["kv_dev"] = torch.empty(kv_self.shape[2:], dtype=torch.float32, device=dev)
         host["x"].copy_(x_new.cpu())
         step(host=host)
         torch.cuda.synchronize()
@@ -401,14 +419,16 @@ def run_ours(a, cfg):
         e1.record()
         torch.cuda.synchronize()
         e2e_value = job_value(ctx_tokens_step, a.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), dev))
-    h2d = T * D * B * H * d * 4 + int(np.prod(x_shape)) * 2
+    h2d = T * D * B * H * d * 4 * (3 if kv_self is not None else 1) + int(np.prod(x_shape)) * 2
     d2h = T * D * B * H * d * 4
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": config_json(cfg, a.workload, world),
+                "config": dict(config_json(cfg, a.workload, world),
+                               **({"self_slot": "current token's exact K/V attended in every call"}
+                                  if kv_self is not None else {})),
                 "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
                 "roofline": roofline(cfg, kernel_name, kern_ms, a.workload),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
