@@ -70,13 +70,19 @@ _decode_2d = _sig("lla_decode_attn_2d", _i, _decode_args + [_vp])
 _decode_ex = _sig("lla_decode_attn_ex", _i, _decode_args + [ctypes.POINTER(DecodeOpts), _vp])
 _flags = _sig("lla_workspace_flags", _i, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp])
 _decode_noalloc = _sig("lla_decode_attn_noalloc", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp])
+_paged_bytes = _sig("lla_paged_store_bytes", _sz, [ctypes.POINTER(CodecDesc), _i])
+_encode_paged = _sig("lla_encode_paged", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _vp])
+_decode_paged = _sig("lla_decode_attn_paged", _i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f,
+                                                   _vp, _vp, _sz, ctypes.POINTER(DecodeOpts), _vp])
 _decode_self = _sig("lla_decode_attn_self", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _sz,
                                                  ctypes.POINTER(DecodeOpts), _vp])
 
 EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy_codec", "lla_codec_get_desc",
             "lla_store_bytes", "lla_encode", "lla_decode_workspace_bytes", "lla_decode_attn",
             "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc",
-            "lla_decode_attn_self"]
+            "lla_decode_attn_self", "lla_paged_store_bytes", "lla_encode_paged", "lla_decode_attn_paged"]
+PAGE_TOKENS = 128
+FLAG_PAGE_INVALID = 4
 
 
 class LLAError(RuntimeError):
@@ -244,10 +250,34 @@ def decode_attn_self(codec, store, batch, max_tokens, layer, loop, q, q_pos, seq
     _check(st, "lla_decode_attn_self")
 
 
+def paged_store_bytes(desc: Desc, num_pages: int) -> int:
+    return int(_paged_bytes(ctypes.byref(desc.c()), num_pages))
+
+
+def encode_paged(codec, x, n, layer_begin, num_layers, seq_idx, tok_idx, pool, num_pages, block_table, max_pages,
+                 batch, stream=None):
+    """lla_encode_paged: write latents into a paged store (pages of PAGE_TOKENS tokens)."""
+    _check(_encode_paged(codec.handle, _ptr(x), n, layer_begin, num_layers, _ptr(seq_idx), _ptr(tok_idx), _ptr(pool),
+                         num_pages, _ptr(block_table), max_pages, batch, _stream(stream)), "lla_encode_paged")
+
+
+def decode_attn_paged(codec, pool, num_pages, block_table, max_pages, batch, layer, loop, q, q_pos, seq_lens, scale,
+                      out, workspace, k_self=None, v_self=None, workspace_bytes=None, stream=None, impl=IMPL_AUTO,
+                      num_ctas=0, events=None):
+    """lla_decode_attn_paged: decode attention over a paged store, optional self slot."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    opts = DecodeOpts(impl, num_ctas, *(events if events is not None else (None, None)))
+    st = _decode_paged(codec.handle, _ptr(pool), num_pages, _ptr(block_table), max_pages, batch, layer, loop, _ptr(q),
+                       _ptr(q_pos), _ptr(seq_lens), _ptr(k_self), _ptr(v_self), float(scale), _ptr(out),
+                       _ptr(workspace), int(workspace_bytes), ctypes.byref(opts), _stream(stream))
+    _check(st, "lla_decode_attn_paged")
+
+
 def raw_decode_status(fn_name, *args) -> int:
     """Call a decode entry point with raw arguments and return its status (for ABI tests)."""
     return {"lla_decode_attn": _decode, "lla_decode_attn_2d": _decode_2d, "lla_decode_attn_ex": _decode_ex,
-            "lla_decode_attn_self": _decode_self}[fn_name](*args)
+            "lla_decode_attn_self": _decode_self, "lla_decode_attn_paged": _decode_paged}[fn_name](*args)
 
 
 def workspace_flags(workspace, stream=None) -> int:

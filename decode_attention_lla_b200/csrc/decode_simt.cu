@@ -18,6 +18,7 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kTile = 128;
+static_assert(kTile == kPageTokens, "a tile of a paged store is one page");
 constexpr int kMaxRv = 256;  // two accumulators per thread
 
 struct SimtParams {
@@ -33,6 +34,7 @@ struct SimtParams {
     uint32_t* flags;
     int B, D, H, T, d, r_k, r_v, max_tokens, max_pos, layer, loop, splits, variant;
     float scale;
+    lla_store_map smap;
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -63,6 +65,10 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(SimtParams p) {
     if (n > p.max_tokens) { n = p.max_tokens; if (tid == 0) atomicOr(p.flags, LLA_FLAG_SEQ_LEN_CLAMPED); }
     if (n > p.max_pos) { n = p.max_pos; if (tid == 0) atomicOr(p.flags, LLA_FLAG_POS_CLAMPED); }
     if (n < 0) n = 0;
+    {
+        const int nu = p.smap.usable_tokens(b, n);
+        if (nu < n) { n = nu; if (tid == 0) atomicOr(p.flags, LLA_FLAG_PAGE_INVALID); }
+    }
     int qp = p.q_pos[b];
     if (qp < 0 || qp >= p.max_pos) {
         qp = qp < 0 ? 0 : p.max_pos - 1;
@@ -92,7 +98,6 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(SimtParams p) {
 
     const size_t row = p.variant == 0 ? size_t(p.H) * (rk + rv) : size_t(rk + rv);
     const size_t hoff = p.variant == 0 ? size_t(h) * (rk + rv) : 0;
-    const uint16_t* base = p.store + (size_t(b) * p.D + p.layer) * size_t(p.max_tokens) * row + hoff;
 
     float m = -INFINITY, l = 0.f, acc0 = 0.f, acc1 = 0.f;
     __syncthreads();
@@ -101,9 +106,11 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(SimtParams p) {
         const int j0 = tile * kTile;
         const int cnt = min(kTile, n - j0);
         const int j = j0 + tid;
+        // the tile's rows are consecutive (a whole page of a paged store)
+        const uint16_t* base = p.store + size_t(p.smap.row_index(b, p.layer, j0, p.D, p.max_tokens)) * row + hoff;
         float s = -INFINITY;
         if (tid < cnt) {
-            const uint16_t* cr = base + size_t(j) * row;
+            const uint16_t* cr = base + size_t(tid) * row;
             for (int a = 0; a < rk; ++a) cT[a * kTile + tid] = bf16_to_f32(cr[a]);
             const float* cs = p.rope_cos + size_t(j) * half;
             const float* sn = p.rope_sin + size_t(j) * half;
@@ -139,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(SimtParams p) {
         l = l * alpha + (red[4] + red[5] + red[6] + red[7]);
         // V side in latent space: acc[a] += sum_j p_j c^V_{j,a}
         {
-            const uint16_t* vb = base + size_t(j0) * row + rk;
+            const uint16_t* vb = base + rk;
             int a = tid;
             if (a < rv) {
                 float v = 0.f;
@@ -212,6 +219,7 @@ lla_status lla_decode_simt(const lla_decode_call& call, int splits_override) {
     p.r_k = ds.r_k;
     p.r_v = ds.r_v;
     p.max_tokens = call.max_tokens;
+    p.smap = call.smap;
     p.max_pos = ds.max_pos;
     p.layer = call.layer;
     p.loop = call.loop;

@@ -148,7 +148,24 @@ struct TcParams {
     float* records;              // [(G + PARTS*B)][4][HC][RV+2]
     uint32_t* status;
     int B, G;
+    // paged store: tile t of sequence b is pool page table[b * max_pages + t] (null: contiguous)
+    const int32_t* table;
+    int max_pages, D, layer;
 };
+
+static_assert(kTile == kPageTokens, "a tile of a paged store is one page");
+
+// TMA coordinates of tile t of sequence b: the token coordinate of its first row and the outer
+// coordinate (sequence, or pool page and layer of a paged store).
+__device__ __forceinline__ void tile_coords(const TcParams& p, int b, int t, int& tok0, int& outer) {
+    if (p.table) {
+        tok0 = 0;
+        outer = __ldg(p.table + size_t(b) * p.max_pages + t) * p.D + p.layer;
+    } else {
+        tok0 = t * kTile;
+        outer = b;
+    }
+}
 
 // The CTAs form G / parts groups of `parts` CTAs; CTA c serves head part c % parts over the
 // tile range of group c / parts, a contiguous share of the flattened (sequence, tile) space.
@@ -304,13 +321,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                             break;
                         mbar_expect_tx(st_full + slot, C::STAGE_BYTES);
                         uint8_t* dst = stage_s + size_t(slot) * C::STAGE_BYTES;
-                        const int tok = wk.t * kTile + ch * C::TOKS;
+                        int tok, outer;
+                        tile_coords(p, wk.b, wk.t, tok, outer);
+                        tok += ch * C::TOKS;
                         if constexpr (C::WIDE) {
-                            tma_load_4d(dst, &maps.m[0], 0, h, tok, wk.b, st_full + slot, pol_stream);
-                            tma_load_4d(dst + C::K0_BYTES, &maps.m[1], 64, h, tok, wk.b, st_full + slot, pol_stream);
-                            tma_load_4d(dst + C::V_OFF, &maps.m[2], C::RK, h, tok, wk.b, st_full + slot, pol_stream);
+                            tma_load_4d(dst, &maps.m[0], 0, h, tok, outer, st_full + slot, pol_stream);
+                            tma_load_4d(dst + C::K0_BYTES, &maps.m[1], 64, h, tok, outer, st_full + slot, pol_stream);
+                            tma_load_4d(dst + C::V_OFF, &maps.m[2], C::RK, h, tok, outer, st_full + slot, pol_stream);
                         } else {
-                            tma_load_4d(dst, &lat_map, 0, h, tok, wk.b, st_full + slot, pol_stream);
+                            tma_load_4d(dst, &lat_map, 0, h, tok, outer, st_full + slot, pol_stream);
                         }
                         __threadfence_block();  // the armed barrier phase precedes the published round
                         issued[slot] = round + 1;
@@ -649,6 +668,7 @@ struct ProParams {
     uint32_t* status;
     int B, D, T, H, DH, RK, RV, HG, NG, HC, GPC, max_tokens, max_pos, layer, loop, variant;
     float scale;
+    lla_store_map smap;
 };
 
 template <class C>
@@ -668,6 +688,8 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
                 if (n > p.max_tokens) { n = p.max_tokens; atomicOr(p.status, LLA_FLAG_SEQ_LEN_CLAMPED); }
                 if (n > p.max_pos) { n = p.max_pos; atomicOr(p.status, LLA_FLAG_POS_CLAMPED); }
                 if (n < 0) n = 0;
+                const int nu = p.smap.usable_tokens(b, n);
+                if (nu < n) { n = nu; atomicOr(p.status, LLA_FLAG_PAGE_INVALID); }
                 p.lens[b] = n;
             }
             const int tiles = (n + kTile - 1) / kTile;
@@ -876,6 +898,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.loop = call.loop;
     pp.variant = c->desc.variant;
     pp.scale = call.scale;
+    pp.smap = call.smap;
     // split records start empty (l = 0); the combine skips them
     LLA_CUDA_TRY(cudaMemsetAsync(pp.records, 0, pp.n_record_floats * sizeof(float), call.stream));
     tc_prologue_kernel<C><<<1 + (B * C::H + 7) / 8, 256, 0, call.stream>>>(pp);
@@ -884,14 +907,20 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).  Per-head
     // rows load whole (r_k + r_v) rows of TOKS tokens; the 2D row loads 64-element panels of
     // 32 tokens in the 128-byte swizzle that the tensor-core operands use.
+    // A paged store is addressed as (row elems, head, token of the page, pool page * D + layer).
     const int h_map = C::TWO_D ? 1 : C::H;
     const size_t row_bytes = size_t(h_map) * C::ROW * 2;  // one token of one layer
     LatMaps maps;
     memset(&maps, 0, sizeof(maps));
-    const void* base = call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
-    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(h_map), cuuint64_t(call.max_tokens), cuuint64_t(B)};
+    const bool paged = call.smap.table != nullptr;
+    const void* base = paged ? static_cast<const void*>(call.store)
+                             : call.store + size_t(call.layer) * call.max_tokens * (row_bytes / 2);
+    cuuint64_t dims[4] = {cuuint64_t(C::ROW), cuuint64_t(h_map),
+                          cuuint64_t(paged ? kPageTokens : call.max_tokens),
+                          paged ? cuuint64_t(call.smap.num_pages) * c->desc.D : cuuint64_t(B)};
     cuuint64_t strides[3] = {cuuint64_t(C::ROW * 2), cuuint64_t(row_bytes),
-                             cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
+                             paged ? cuuint64_t(row_bytes) * kPageTokens
+                                   : cuuint64_t(row_bytes) * call.max_tokens * c->desc.D};
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     auto encode = [&](CUtensorMap* m, uint32_t box_elems, uint32_t box_toks, CUtensorMapSwizzle swz) {
         cuuint32_t box[4] = {box_elems, 1u, box_toks, 1u};
@@ -921,6 +950,10 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tp.status = pp.status;
     tp.B = B;
     tp.G = G;
+    tp.table = call.smap.table;
+    tp.max_pages = call.smap.max_pages;
+    tp.D = c->desc.D;
+    tp.layer = call.layer;
     void (*kernel)(const LatMaps, TcParams);
     if constexpr (C::TWO_D) kernel = tc2d_decode_kernel<C>;
     else kernel = tc_decode_kernel<C>;

@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     if (round > 0 && !(ok = mbar_wait(k_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 23)))
                         break;
                     mbar_expect_tx(k_full + slot, C::K_SLOT);
-                    tma_load_4d(k_s + size_t(slot) * C::K_SLOT, &lat_map, 0, 0, wk.t * kTile + q * C::QTOK, wk.b,
+                    int tok, outer;
+                    tile_coords(p, wk.b, wk.t, tok, outer);
+                    tma_load_4d(k_s + size_t(slot) * C::K_SLOT, &lat_map, 0, 0, tok + q * C::QTOK, outer,
                                 k_full + slot, pol_stream);
                     __threadfence_block();  // the armed barrier phase precedes the published round
                     k_issued[slot] = round + 1;
@@ -205,6 +207,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             uint32_t vk_n = 0;
             bool ok = true;
             for (; wk.valid() && ok; wk.next()) {
+                int vtok, vouter;
+                tile_coords(p, wk.b, wk.t, vtok, vouter);
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t slot = vk_n % C::NV, round = vk_n / C::NV;
                     if (round > 0 && !(ok = mbar_wait(v_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 27)))
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
 #pragma unroll
                     for (int pn = 0; pn < C::V_PANELS; ++pn)
                         tma_load_4d(v_s + size_t(slot) * C::V_SLOT + pn * C::PANEL, &lat_map, C::RK + 64 * pn, 0,
-                                    wk.t * kTile + q * C::QTOK, wk.b, v_full + slot, pol_stream);
+                                    vtok + q * C::QTOK, vouter, v_full + slot, pol_stream);
                     __threadfence_block();
                     v_issued[slot] = round + 1;
                     ++vk_n;

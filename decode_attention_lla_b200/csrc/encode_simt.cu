@@ -31,6 +31,7 @@ struct EncodeParams {
     const float* bias_k;
     const float* bias_v;
     int n, layer_begin, num_layers, H, S, r_k, r_v, variant, batch, max_tokens, D;
+    lla_store_map smap;
 };
 
 __global__ void __launch_bounds__(kThreads) encode_simt_kernel(EncodeParams p) {
@@ -94,8 +95,10 @@ __global__ void __launch_bounds__(kThreads) encode_simt_kernel(EncodeParams p) {
     if (i >= p.n) return;
     const int sq = p.seq_idx[i], tk = p.tok_idx[i];
     if (sq < 0 || sq >= p.batch || tk < 0 || tk >= p.max_tokens) return;
+    const long long ri = p.smap.row_index(sq, layer, tk, p.D, p.max_tokens);
+    if (ri < 0) return;  // a page index out of range: not written
     const size_t row = p.variant == 0 ? size_t(p.H) * (p.r_k + p.r_v) : size_t(p.r_k + p.r_v);
-    uint16_t* dst = p.store + ((size_t(sq) * p.D + layer) * p.max_tokens + tk) * row +
+    uint16_t* dst = p.store + size_t(ri) * row +
                     (p.variant == 0 ? size_t(h) * (p.r_k + p.r_v) : 0) + (axis == 0 ? 0 : p.r_k);
 #pragma unroll
     for (int u = 0; u < kAcc; ++u) {
@@ -111,19 +114,20 @@ __global__ void __launch_bounds__(kThreads) encode_simt_kernel(EncodeParams p) {
 
 lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                              const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
-                             int max_tokens, cudaStream_t stream) {
+                             int max_tokens, cudaStream_t stream, const lla_store_map& smap) {
     // the tensor-core kernel where it applies (TMA needs 16-byte aligned rows and stacks)
     if ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(store) & 15) == 0) {
-        const lla_status st =
-            lla_encode_tc(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+        const lla_status st = lla_encode_tc(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch,
+                                            max_tokens, stream, smap);
         if (st != LLA_ERR_UNSUPPORTED_SHAPE) return st;
     }
-    return lla_encode_simt(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+    return lla_encode_simt(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream,
+                           smap);
 }
 
 lla_status lla_encode_simt(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                            const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
-                           int max_tokens, cudaStream_t stream) {
+                           int max_tokens, cudaStream_t stream, const lla_store_map& smap) {
     const lla_codec_desc& ds = c->desc;
     if (ds.r_k > kMaxR || ds.r_v > kMaxR) return LLA_ERR_UNSUPPORTED_SHAPE;
     EncodeParams p;
@@ -146,6 +150,7 @@ lla_status lla_encode_simt(const lla_codec* c, const uint16_t* x, int n, int lay
     p.batch = batch;
     p.max_tokens = max_tokens;
     p.D = ds.D;
+    p.smap = smap;
     const int rmax = ds.r_k > ds.r_v ? ds.r_k : ds.r_v;
     const size_t smem = size_t(rmax) * kK * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(encode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));

@@ -66,6 +66,7 @@ struct EncParams {
     uint32_t* status;
     int n, layer_begin, num_layers, Hg, S, D, batch, max_tokens;
     size_t row;  // elements per (sequence, layer, token) row of the store
+    lla_store_map smap;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -185,9 +186,10 @@ __global__ void __launch_bounds__(kThreads) encode_tc_kernel(const __grid_consta
             sq = p.seq_idx[i];
             tk = p.tok_idx[i];
         }
-        const bool write = ok && i < p.n && sq >= 0 && sq < p.batch && tk >= 0 && tk < p.max_tokens;
-        uint16_t* dst = p.store + ((size_t(sq < 0 ? 0 : sq) * p.D + layer) * p.max_tokens + (tk < 0 ? 0 : tk)) * p.row +
-                        size_t(h) * (C::RK + C::RV);
+        bool write = ok && i < p.n && sq >= 0 && sq < p.batch && tk >= 0 && tk < p.max_tokens;
+        const long long ri = write ? p.smap.row_index(sq, layer, tk, p.D, p.max_tokens) : 0;
+        write = write && ri >= 0;  // a page index out of range: not written
+        uint16_t* dst = p.store + size_t(ri < 0 ? 0 : ri) * p.row + size_t(h) * (C::RK + C::RV);
         const float* bk = p.bias_k + (size_t(layer) * p.Hg + h) * C::RK;
         const float* bv = p.bias_v + (size_t(layer) * p.Hg + h) * C::RV;
 #pragma unroll
@@ -271,7 +273,7 @@ bool make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int rank, con
 template <class C>
 lla_status run_encode(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                       const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const lla_store_map& smap) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LLA_ERR_CUDA;
     const lla_codec_desc& ds = c->desc;
@@ -312,6 +314,7 @@ lla_status run_encode(const lla_codec* c, const uint16_t* x, int n, int layer_be
     p.batch = batch;
     p.max_tokens = max_tokens;
     p.row = size_t(ds.r_k + ds.r_v) * Hg;
+    p.smap = smap;
     LLA_CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     dim3 grid((n + kTok - 1) / kTok, num_layers * Hg);
     encode_tc_kernel<C><<<grid, kThreads, C::SMEM, stream>>>(xmap, wkmap, wvmap, p);
@@ -324,14 +327,17 @@ lla_status run_encode(const lla_codec* c, const uint16_t* x, int n, int layer_be
 // Tensor-core encode for the codec shapes it is built for; LLA_ERR_UNSUPPORTED_SHAPE otherwise.
 lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                          const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const lla_store_map& smap) {
     const lla_codec_desc& d = c->desc;
     if (c->S % kKc != 0 || !c->status) return LLA_ERR_UNSUPPORTED_SHAPE;
     if (d.r_k == 16 && d.r_v == 32)
-        return run_encode<ECfg<16, 32>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+        return run_encode<ECfg<16, 32>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens,
+                                        stream, smap);
     if (d.r_k == 96 && d.r_v == 160)
-        return run_encode<ECfg<96, 160>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+        return run_encode<ECfg<96, 160>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch,
+                                         max_tokens, stream, smap);
     if (d.r_k == 64 && d.r_v == 128)
-        return run_encode<ECfg<64, 128>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch, max_tokens, stream);
+        return run_encode<ECfg<64, 128>>(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, store, batch,
+                                         max_tokens, stream, smap);
     return LLA_ERR_UNSUPPORTED_SHAPE;
 }

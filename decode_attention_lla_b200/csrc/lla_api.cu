@@ -92,6 +92,10 @@ size_t lla_store_bytes(const lla_codec_desc* d, int batch, int max_tokens) {
     return size_t(batch) * size_t(d->D) * size_t(max_tokens) * per * 2;
 }
 
+size_t lla_paged_store_bytes(const lla_codec_desc* d, int num_pages) {
+    return lla_store_bytes(d, num_pages, kPageTokens);  // a page holds kPageTokens tokens of every layer
+}
+
 lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const float* w_down_k,
                             const float* w_down_v, const float* w_up_k, const float* w_up_v,
                             const float* mu_k, const float* mu_v, void* stream_) {
@@ -217,6 +221,24 @@ lla_status lla_encode(const lla_codec* c, const uint16_t* x, int n, int layer_be
                              static_cast<cudaStream_t>(stream));
 }
 
+lla_status lla_encode_paged(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
+                            const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* pool, int num_pages,
+                            const int32_t* block_table, int max_pages, int batch, void* stream) {
+    if (!c || n < 0 || batch < 0 || num_pages < 1 || max_pages < 1) return LLA_ERR_INVALID_ARG;
+    if (max_pages > (1 << 30) / kPageTokens) return LLA_ERR_INVALID_ARG;
+    if (layer_begin < 0 || num_layers < 1 || layer_begin + num_layers > c->desc.D) return LLA_ERR_INVALID_ARG;
+    if (n == 0) return LLA_OK;
+    if (!x || !seq_idx || !tok_idx || !pool || !block_table) return LLA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(pool) || !aligned4(seq_idx) || !aligned4(tok_idx) || !aligned4(block_table))
+        return LLA_ERR_ALIGNMENT;
+    lla_store_map smap;
+    smap.table = block_table;
+    smap.max_pages = max_pages;
+    smap.num_pages = num_pages;
+    return lla_encode_launch(c, x, n, layer_begin, num_layers, seq_idx, tok_idx, pool, batch,
+                             max_pages * kPageTokens, static_cast<cudaStream_t>(stream), smap);
+}
+
 size_t lla_decode_workspace_bytes(const lla_codec* c, int batch, int max_tokens) {
     if (!c || batch < 0 || max_tokens < 0) return 0;
     size_t a = lla_simt_workspace_bytes(c, batch, max_tokens);
@@ -231,7 +253,8 @@ static lla_status decode_common(int want_variant, const lla_codec* c, const uint
                                 int max_tokens, int layer, int loop, const float* q, const int32_t* q_pos,
                                 const int32_t* seq_lens, float scale, float* out, void* workspace,
                                 size_t workspace_bytes, const lla_decode_opts* opts, void* stream,
-                                const float* k_self = nullptr, const float* v_self = nullptr) {
+                                const float* k_self = nullptr, const float* v_self = nullptr,
+                                const lla_store_map& smap = lla_store_map()) {
     if (!c || c->desc.variant != want_variant) return LLA_ERR_INVALID_ARG;
     if (batch < 0 || max_tokens < 0 || layer < 0 || layer >= c->desc.D || loop < 0 || loop >= c->desc.T)
         return LLA_ERR_INVALID_ARG;
@@ -270,6 +293,7 @@ static lla_status decode_common(int want_variant, const lla_codec* c, const uint
     }
     call.k_self = k_self;
     call.v_self = v_self;
+    call.smap = smap;
     LLA_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(lla_ws_header), call.stream));
     if (max_tokens == 0) {
         // no cached token: the softmax is empty (zero output) or the self slot alone (its value)
@@ -316,6 +340,22 @@ lla_status lla_decode_attn_self(const lla_codec* c, const uint16_t* store, int b
     if (batch > 0 && (!k_self || !v_self)) return LLA_ERR_INVALID_ARG;
     return decode_common(c->desc.variant, c, store, batch, max_tokens, layer, loop, q, q_pos, seq_lens, scale, out,
                          workspace, workspace_bytes, opts, stream, k_self, v_self);
+}
+
+lla_status lla_decode_attn_paged(const lla_codec* c, const uint16_t* pool, int num_pages, const int32_t* block_table,
+                                 int max_pages, int batch, int layer, int loop, const float* q, const int32_t* q_pos,
+                                 const int32_t* seq_lens, const float* k_self, const float* v_self, float scale,
+                                 float* out, void* workspace, size_t workspace_bytes, const lla_decode_opts* opts,
+                                 void* stream) {
+    if (!c || num_pages < 1 || max_pages < 1 || max_pages > (1 << 30) / kPageTokens) return LLA_ERR_INVALID_ARG;
+    if (batch > 0 && !block_table) return LLA_ERR_INVALID_ARG;
+    if (block_table && !aligned4(block_table)) return LLA_ERR_ALIGNMENT;
+    lla_store_map smap;
+    smap.table = block_table;
+    smap.max_pages = max_pages;
+    smap.num_pages = num_pages;
+    return decode_common(c->desc.variant, c, pool, batch, max_pages * kPageTokens, layer, loop, q, q_pos, seq_lens,
+                         scale, out, workspace, workspace_bytes, opts, stream, k_self, v_self, smap);
 }
 
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {

@@ -46,6 +46,34 @@ struct lla_ws_header {
 enum : uint32_t {
     LLA_FLAG_SEQ_LEN_CLAMPED = 1u,
     LLA_FLAG_POS_CLAMPED = 2u,
+    LLA_FLAG_PAGE_INVALID = 4u,
+};
+
+// Where the rows of a latent store live.  Contiguous: [batch][D][max_tokens][row].  Paged: a
+// pool of pages [num_pages][D][kPageTokens][row]; token j of sequence b sits in pool page
+// table[b * max_pages + j / kPageTokens], slot j % kPageTokens.
+constexpr int kPageTokens = 128;
+struct lla_store_map {
+    const int32_t* table = nullptr;  // null: contiguous
+    int max_pages = 0;
+    int num_pages = 0;
+    // row index of (b, layer, token), or -1 when the token's page index is out of range
+    __host__ __device__ long long row_index(int b, int layer, int tok, int D, int max_tokens) const {
+        if (!table) return (static_cast<long long>(b) * D + layer) * max_tokens + tok;
+        const int pg = table[static_cast<size_t>(b) * max_pages + tok / kPageTokens];
+        if (pg < 0 || pg >= num_pages) return -1;
+        return (static_cast<long long>(pg) * D + layer) * kPageTokens + tok % kPageTokens;
+    }
+    // tokens of sequence b usable with this map: n, cut before its first page that is out of
+    // range (paged stores only)
+    __device__ int usable_tokens(int b, int n) const {
+        if (!table) return n;
+        for (int pg = 0; pg * kPageTokens < n; ++pg) {
+            const int e = table[static_cast<size_t>(b) * max_pages + pg];
+            if (e < 0 || e >= num_pages) return pg * kPageTokens;
+        }
+        return n;
+    }
 };
 
 // Common decode-call parameters after host validation.
@@ -65,6 +93,7 @@ struct lla_decode_call {
     cudaEvent_t ev_end = nullptr;
     const float* k_self = nullptr;   // optional self slot: the current token's exact loop-t
     const float* v_self = nullptr;   // key (pre-RoPE) and value, [batch][H][d_head]
+    lla_store_map smap;              // paged store (max_tokens = max_pages * kPageTokens)
 };
 
 // ---- bf16 helpers ---------------------------------------------------------
@@ -94,14 +123,15 @@ struct lla_tc_ranges {
 lla_status lla_combine_tc(const lla_decode_call& call, const float* records, const lla_tc_ranges& r);
 lla_status lla_encode_launch(const lla_codec* c, const uint16_t* x, int n, int layer_begin,
                              int num_layers, const int32_t* seq_idx, const int32_t* tok_idx,
-                             uint16_t* store, int batch, int max_tokens, cudaStream_t stream);
+                             uint16_t* store, int batch, int max_tokens, cudaStream_t stream,
+                             const lla_store_map& smap = lla_store_map());
 lla_status lla_build_phi_tiles(lla_codec* c, cudaStream_t stream);
 lla_status lla_encode_simt(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                            const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch,
-                           int max_tokens, cudaStream_t stream);
+                           int max_tokens, cudaStream_t stream, const lla_store_map& smap);
 lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer_begin, int num_layers,
                          const int32_t* seq_idx, const int32_t* tok_idx, uint16_t* store, int batch, int max_tokens,
-                         cudaStream_t stream);
+                         cudaStream_t stream, const lla_store_map& smap);
 
 int lla_num_sms();
 

@@ -200,6 +200,55 @@ lla_status lla_decode_attn_ex(const lla_codec* codec, const uint16_t* store, int
                               void* stream);
 
 /*
+ * Paged latent stores.  A pool of pages, each holding LLA_PAGE_TOKENS consecutive
+ * tokens of one sequence for every layer:
+ *   per-head: pool[num_pages][D][LLA_PAGE_TOKENS][H][r_k + r_v]
+ *   LLA-2D:   pool[num_pages][D][LLA_PAGE_TOKENS][r_k + r_v]
+ * and a block table, device int32 [batch][max_pages]: token j of sequence b
+ * lives in pool page block_table[b][j / LLA_PAGE_TOKENS], slot
+ * j % LLA_PAGE_TOKENS.  A sequence's logical capacity is
+ * max_pages * LLA_PAGE_TOKENS tokens; its pages need not be contiguous or in
+ * order, and entries past its length are not read.  The method is unchanged
+ * [LLA §3 eqs. (2)-(3)]: only where a latent row is kept differs (serving
+ * systems page their caches; the paper's store is the contiguous layout).
+ */
+#define LLA_PAGE_TOKENS 128
+
+/* Bytes of a pool of num_pages pages (0 for an invalid description). */
+size_t lla_paged_store_bytes(const lla_codec_desc* desc, int num_pages);
+
+/*
+ * lla_encode_paged — lla_encode into a paged store.  Rows whose sequence,
+ *   token (>= max_pages * LLA_PAGE_TOKENS) or page index (outside
+ *   [0, num_pages)) is out of range are not written.
+ *   pool        device bf16, lla_paged_store_bytes(desc, num_pages) bytes
+ *   block_table device int32 [batch][max_pages]
+ */
+lla_status lla_encode_paged(const lla_codec* codec, const uint16_t* x, int n,
+                            int layer_begin, int num_layers,
+                            const int32_t* seq_idx, const int32_t* tok_idx,
+                            uint16_t* pool, int num_pages, const int32_t* block_table,
+                            int max_pages, int batch, void* stream);
+
+/*
+ * lla_decode_attn_paged — decode attention (either codec variant) over a paged
+ *   store, with an optional self slot (k_self and v_self both NULL: none; see
+ *   lla_decode_attn_self).  Results equal those of the contiguous store
+ *   holding the same rows.  seq_lens[b] <= max_pages * LLA_PAGE_TOKENS; a
+ *   block-table entry outside [0, num_pages) among a sequence's pages cuts the
+ *   sequence before that page and sets LLA_FLAG_PAGE_INVALID (4) in the
+ *   workspace status.  The workspace is sized by
+ *   lla_decode_workspace_bytes(codec, batch, max_pages * LLA_PAGE_TOKENS).
+ */
+lla_status lla_decode_attn_paged(const lla_codec* codec, const uint16_t* pool, int num_pages,
+                                 const int32_t* block_table, int max_pages, int batch,
+                                 int layer, int loop, const float* q, const int32_t* q_pos,
+                                 const int32_t* seq_lens, const float* k_self,
+                                 const float* v_self, float softmax_scale, float* out,
+                                 void* workspace, size_t workspace_bytes,
+                                 const lla_decode_opts* opts, void* stream);
+
+/*
  * lla_decode_attn_self — decode attention with the current token as a self slot
  *   [LLA §3 eq. (2)-(3)]: a token's latent is written only after its last loop
  *   (eq. (2) encodes the whole loop stack), so while it is being decoded its
