@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--mode", choices=["decode", "encode"], default="decode",
                     help="encode: time prefill encoding of teacher stacks instead of the decode step")
     ap.add_argument("--encode-tokens", type=int, default=4096, help="tokens per encode call (encode mode)")
+    ap.add_argument("--paged", action="store_true",
+                    help="latent store as a pool of 128-token pages in shuffled order with a block table")
     ap.add_argument("--self-slot", action="store_true",
                     help="decode calls attend to the current token's exact K/V as well (lla_decode_attn_self)")
     return ap.parse_args()
@@ -306,7 +308,14 @@ def run_ours(a, cfg):
     codec = lla.Codec(desc, codec_np["w_down_k"], codec_np["w_down_v"], codec_np["w_up_k"], codec_np["w_up_v"],
                       codec_np["mu_k"], codec_np["mu_v"])
     del codec_np
-    nbytes = lla.store_bytes(desc, B, cap)
+    pages = (cap + lla.PAGE_TOKENS - 1) // lla.PAGE_TOKENS  # per sequence
+    table = None
+    if a.paged:  # every sequence's pages scattered over the pool in a seeded random order
+        nbytes = lla.paged_store_bytes(desc, B * pages)
+        perm = syn.rng(tag + "/pages").permutation(B * pages).astype(np.int32).reshape(B, pages)
+        table = torch.from_numpy(perm).to(dev)
+    else:
+        nbytes = lla.store_bytes(desc, B, cap)
     store = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
     syn.fill_gaussian_bf16_(store, tag + "/store")
     q_all = torch.empty(T, D, B, H, d, dtype=torch.float32, device=dev)
@@ -324,14 +333,24 @@ def run_ours(a, cfg):
     lens = torch.full((B,), N, dtype=torch.int32, device=dev)
     qpos = torch.full((B,), N, dtype=torch.int32, device=dev)
     out = torch.empty(B, H, d, dtype=torch.float32, device=dev)
-    ws = torch.empty(codec.workspace_bytes(B, cap), dtype=torch.uint8, device=dev)
+    ws = torch.empty(codec.workspace_bytes(B, pages * lla.PAGE_TOKENS if a.paged else cap), dtype=torch.uint8,
+                     device=dev)
     impl = {"auto": lla.IMPL_AUTO, "simt": lla.IMPL_SIMT, "tc": lla.IMPL_TC}[a.kernel]
     scale = 1.0 / math.sqrt(d)
-    decode = lla.decode_attn if cfg["variant"] == 0 else lla.decode_attn_2d
     kernel_name = a.kernel
+    def decode_call(layer, t, q, ks, vs, impl, ev):
+        if table is not None:
+            lla.decode_attn_paged(codec, store, B * pages, table, pages, B, layer, t, q, qpos, lens, scale, out, ws,
+                                  k_self=ks, v_self=vs, impl=impl, events=ev)
+        elif ks is not None:
+            lla.decode_attn_self(codec, store, B, cap, layer, t, q, qpos, lens, ks, vs, scale, out, ws, impl=impl,
+                                 events=ev)
+        else:
+            lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl, events=ev)
+
     if a.kernel == "auto":  # find which kernel "auto" runs
         try:
-            lla.decode_attn(codec, store, B, cap, 0, 0, q_all[0, 0], qpos, lens, scale, out, ws, impl=lla.IMPL_TC)
+            decode_call(0, 0, q_all[0, 0], None, None, lla.IMPL_TC, None)
             kernel_name = "tc"
         except lla.LLAError:
             kernel_name = "simt"
@@ -346,22 +365,23 @@ def run_ours(a, cfg):
                     q = host["q_dev"]
                     q.copy_(host["q"][t, layer], non_blocking=True)
                 ev = events[k] if events is not None else None
-                if kv_self is None:
-                    lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl,
-                                    events=ev)
-                else:
+                ks = vs = None
+                if kv_self is not None:
                     kv = kv_self[t, layer]
                     if host is not None:
                         kv = host["kv_dev"]
                         kv.copy_(host["kv"][t, layer], non_blocking=True)
-                    lla.decode_attn_self(codec, store, B, cap, layer, t, q, qpos, lens, kv[0], kv[1], scale, out,
-                                         ws, impl=impl, events=ev)
+                    ks, vs = kv[0], kv[1]
+                decode_call(layer, t, q, ks, vs, impl, ev)
                 if host is not None:
                     host["out"][t, layer].copy_(out, non_blocking=True)
                 k += 1
         if host is not None:
             x_new.copy_(host["x"], non_blocking=True)
-        lla.encode(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B, cap)
+        if table is not None:
+            lla.encode_paged(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B * pages, table, pages, B)
+        else:
+            lla.encode(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B, cap)
 
     for _ in range(a.warmup):
         step()
@@ -428,7 +448,9 @@ def run_ours(a, cfg):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(config_json(cfg, a.workload, world),
                                **({"self_slot": "current token's exact K/V attended in every call"}
-                                  if kv_self is not None else {})),
+                                  if kv_self is not None else {}),
+                               **({"store": f"paged: {pages} pages of {lla.PAGE_TOKENS} tokens per sequence, "
+                                            "shuffled over the pool"} if table is not None else {})),
                 "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
                 "roofline": roofline(cfg, kernel_name, kern_ms, a.workload),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -450,6 +472,8 @@ def main():
     if a.batch or a.layers:
         cfg.update(batch=a.batch or cfg["batch"], D=a.layers or cfg["D"])
         a.workload = f"{a.workload}[batch={cfg['batch']},layers={cfg['D']}]"
+    if getattr(a, "paged", False) or getattr(a, "self_slot", False):
+        a.workload += "[" + ",".join(k for k, on in (("paged", a.paged), ("self-slot", a.self_slot)) if on) + "]"
     if a.impl == "reference":
         return run_reference(a, cfg)
     if a.mode == "encode":

@@ -18,17 +18,20 @@
 // in latent space: acc += p_j c^V_j.  The split-combine kernel lifts acc.
 //
 // Kernel structure (one CTA per SM, persistent over a flattened range of
-// (head part, sequence, 128-token tile) work):
-//   warp 0      TMA producer: M_q image per (sequence, head part), Phi tile
-//               per tile, latent tiles per (tile, head, token chunk) into a
-//               ring of shared-memory stages (mbarrier full/empty pairs).
-//   warp 1      TMEM allocator and MMA issuer: per tile and head group,
-//               d/16 tcgen05.mma (M=128, N=NG, K=16, fp16 in, fp32 out) into
-//               one of two TMEM buffers, committed to an mbarrier.
-//   warps 2-9   compute: thread = token row (its TMEM lane); two warps share a
-//               lane quarter and split the heads of each group.  Each warp
-//               keeps (m, l, acc) per head for its 32 rows and writes one
-//               record per (segment, quarter, head) for the combine kernel.
+// (head part, sequence, 128-token tile) work), per-head latents:
+//   warp 0      TMA producer of latent stages: per (tile, head, token chunk) a box
+//               of (r_k + r_v) x 1 head x TOKS tokens (wide rows: three panels, the
+//               c^K ones swizzled) into a ring of shared-memory stages.
+//   warp 1      TMEM allocator and MMA issuer: per tile and head group, d/16
+//               tcgen05.mma (M=128, N=NG, K=16, fp16 in, fp32 out) into a ring of
+//               TMEM buffers, committed to mbarriers.
+//   warp 2      (narrow rows) TMA producer of the M_q image per (sequence, head
+//               part) and the Phi tile per tile; with wide rows warp 0 does this.
+//   the rest    compute: thread = token row (its TMEM lane); the warps of a lane
+//               quarter split the heads of each group.  Each keeps (m, l, acc) per
+//               head for its 32 rows and writes one record per (segment, quarter,
+//               head) for the combine kernel.
+// The LLA-2D kernel (decode_tc2d.cuh) shares the walk, the prologue and the records.
 // Every wait is bounded (see sm100.cuh); a timeout sets a status bit.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -106,7 +109,10 @@ struct Cfg : HeadGroups<DH_, RK_, RV_, H_, WIDE_ ? 1 : 8> {
     // compute warps: WPQ per TMEM lane quarter, each taking HG / WPQ heads of every group
     static constexpr int WPQ = WIDE ? 1 : (HG >= 4 ? 4 : HG);
     static constexpr int NCW = 4 * WPQ;
-    static constexpr int THREADS = 32 * (2 + NCW);
+    // warps: latent-stage producer, MMA issuer, (narrow rows) M_q/Phi producer, compute
+    static constexpr bool PHI_WARP = !WIDE;
+    static constexpr int CW0 = PHI_WARP ? 3 : 2;
+    static constexpr int THREADS = 32 * (CW0 + NCW);
     static constexpr int HPW = HC / WPQ;  // heads per compute warp
     // one stage per (head, token chunk), read by that head's warp of each quarter in the chunk
     static constexpr int STAGES_PER_TILE = HC * CHUNKS;
@@ -287,32 +293,44 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     TileWalker wk;
     wk.init(p.P, p.B, p.G, blockIdx.x, C::PARTS);
 
+    // M_q image on a sequence change and the tile's Phi: issued by the elected thread of the
+    // warp that owns them
+    uint32_t phi_n = 0, mq_n = 0;
+    int mq_key = -1;
+    auto phi_mq_step = [&]() -> bool {
+        const uint64_t pol_keep = policy_evict_last();
+        const int key = wk.key();
+        if (key != mq_key) {
+            if (mq_n > 0 && !mbar_wait(mq_empty, (mq_n - 1) & 1, p.status, kFlagTimeout, 1)) return false;
+            mbar_expect_tx(mq_full, C::MQ_BYTES);
+            const uint8_t* src = p.mq + (size_t(wk.p) * p.B + wk.b) * C::MQ_BYTES;
+            for (int off = 0; off < C::MQ_BYTES; off += 32768) {
+                const int n = C::MQ_BYTES - off < 32768 ? C::MQ_BYTES - off : 32768;
+                bulk_g2s(mq_s + off, src + off, n, mq_full, pol_keep);
+            }
+            ++mq_n;
+            mq_key = key;
+        }
+        if (phi_n > 0 && !mbar_wait(phi_empty, (phi_n - 1) & 1, p.status, kFlagTimeout, 2)) return false;
+        mbar_expect_tx(phi_full, C::PHI_BYTES);
+        bulk_g2s(phi_s, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES, phi_full, pol_keep);
+        ++phi_n;
+        return true;
+    };
+    auto phi_mq_drain = [&]() {
+        if (phi_n > 0) mbar_wait(phi_full, (phi_n - 1) & 1, p.status, kFlagTimeout, 5);
+        if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
+    };
+
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ latent stage producer
         if (elect_one()) {
             prefetch_tensormap(&lat_map);
             const uint64_t pol_stream = policy_evict_first();
-            const uint64_t pol_keep = policy_evict_last();
-            uint32_t stage_k = 0, phi_n = 0, mq_n = 0;
-            int prev_key = -1;
+            uint32_t stage_k = 0;
             bool ok = true;
             for (; wk.valid() && ok; wk.next()) {
-                const int key = wk.key();
-                if (key != prev_key) {
-                    if (mq_n > 0 && !(ok = mbar_wait(mq_empty, (mq_n - 1) & 1, p.status, kFlagTimeout, 1))) break;
-                    mbar_expect_tx(mq_full, C::MQ_BYTES);
-                    const uint8_t* src = p.mq + (size_t(wk.p) * p.B + wk.b) * C::MQ_BYTES;
-                    for (int off = 0; off < C::MQ_BYTES; off += 32768) {
-                        const int n = C::MQ_BYTES - off < 32768 ? C::MQ_BYTES - off : 32768;
-                        bulk_g2s(mq_s + off, src + off, n, mq_full, pol_keep);
-                    }
-                    ++mq_n;
-                    prev_key = key;
-                }
-                if (phi_n > 0 && !(ok = mbar_wait(phi_empty, (phi_n - 1) & 1, p.status, kFlagTimeout, 2))) break;
-                mbar_expect_tx(phi_full, C::PHI_BYTES);
-                bulk_g2s(phi_s, p.phi_tiles + size_t(wk.t) * (C::PHI_BYTES / 2), C::PHI_BYTES, phi_full, pol_keep);
-                ++phi_n;
+                if (!C::PHI_WARP && !(ok = phi_mq_step())) break;
                 for (int hl = 0; hl < C::HC && ok; ++hl) {
                     const int h = wk.p * C::HC + hl;
                     for (int ch = 0; ch < C::CHUNKS; ++ch) {
@@ -342,8 +360,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last issue into slot s
                 mbar_wait(st_full + s, (last / C::NST) & 1, p.status, kFlagTimeout, 4);
             }
-            if (phi_n > 0) mbar_wait(phi_full, (phi_n - 1) & 1, p.status, kFlagTimeout, 5);
-            if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
+            if (!C::PHI_WARP) phi_mq_drain();
+        }
+    } else if (C::PHI_WARP && warp == 2) {
+        // ------------------------------------------------------------ M_q and Phi producer
+        // (its own warp, so the next tile's Phi goes out as soon as its buffer is free rather
+        // than behind the current tile's latent stages)
+        if (elect_one()) {
+            bool ok = true;
+            for (; wk.valid() && ok; wk.next()) ok = phi_mq_step();
+            phi_mq_drain();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -395,7 +421,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         }
     } else {
         // ------------------------------------------------------------ compute warps
-        const int cw = warp - 2;
+        const int cw = warp - C::CW0;
         const int qd = warp & 3;        // TMEM lane quarter = token rows [32 qd, 32 qd + 32)
         const int hf = cw >> 2;         // which of the WPQ warps of this quarter
         const int row = 32 * qd + lane;  // tile row of this thread
