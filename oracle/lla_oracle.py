@@ -57,6 +57,7 @@ __all__ = [
     "lla_decode",
     "lla_decode_2d",
     "encode_2d",
+    "full_decode",
 ]
 
 
@@ -294,4 +295,29 @@ def lla_decode_2d(q, cK, cV, muK, WupK, muV, WupV, loop, seq_lens, q_pos, scale,
             out[b, h] = lla_decode_head(q[b, h], cK[b, :n], cV[b, :n],
                                         muK[loop, h], WupK[loop, h], muV[loop, h], WupV[loop, h],
                                         float(q_pos[b]), scale, base, ks, vs)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Comparator: decode over a full (uncompressed) K/V cache
+# ---------------------------------------------------------------------------
+
+def full_decode(q, K_rot, V, seq_lens, q_pos, scale, base):
+    """Decode attention over a full cache, the comparator of the latent store.
+
+    The "fast path" the summary page contrasts with the latent path keeps, for
+    each cached token, the loop-t key and value themselves [LLA summary,
+    "Serving Capacity"; LLA §3, "Teacher cache"]; keys are cached already
+    rotated at their positions, so only the query is rotated here.
+    q [B, H, d] pre-RoPE; K_rot, V [B, N, H, d]; returns out [B, H, d].
+    """
+    q = np.asarray(q, np.float64)
+    B, H, d = q.shape
+    out = np.zeros((B, H, np.asarray(V).shape[-1]), np.float64)
+    for b in range(B):
+        n = int(seq_lens[b])
+        for h in range(H):
+            out[b, h] = softmax_attention(apply_rope(q[b, h], float(q_pos[b]), base),
+                                          np.asarray(K_rot[b, :n, h], np.float64),
+                                          np.asarray(V[b, :n, h], np.float64), scale)
     return out

@@ -27,6 +27,7 @@ PIN_TESTS = [
     pins.test_softmax_special_cases,
     pins.test_self_slot_with_empty_cache_is_its_value,
     pins.test_self_slot_matches_sdpa_over_the_appended_token,
+    pins.test_full_cache_decode_equals_lla_on_the_reconstructed_cache,
     lambda: pins.test_vectorised_oracle_matches_brute_force(dict(T=2, d=4, rk=2, rv=3, n=8, H=2, B=2)),
 ]
 

@@ -271,6 +271,28 @@ def test_self_slot_matches_sdpa_over_the_appended_token():
     assert np.abs(got - (p / p.sum()) @ V).max() < 1e-12
 
 
+def test_full_cache_decode_equals_lla_on_the_reconstructed_cache():
+    """The comparator over the cache a fast path would build (keys reconstructed and rotated at
+    their positions, values reconstructed) gives the LLA result; and it is SDPA per head."""
+    B, n, H, d, rk, rv, T, t = 2, 30, 3, 16, 4, 6, 3, 1
+    cK = syn.gaussian("pin/full/cK", (B, n, H, rk))
+    cV = syn.gaussian("pin/full/cV", (B, n, H, rv))
+    WK, WV = syn.gaussian("pin/full/WK", (H, T, d, rk), 0.3), syn.gaussian("pin/full/WV", (H, T, d, rv), 0.3)
+    muK, muV = syn.gaussian("pin/full/muK", (H, T, d)), syn.gaussian("pin/full/muV", (H, T, d))
+    q = syn.gaussian("pin/full/q", (B, H, d))
+    lens, qpos = np.array([n, 17]), np.array([n, 40])
+    K = np.einsum("bnha,hda->bnhd", cK, WK[:, t]) + muK[None, None, :, t]
+    V = np.einsum("bnha,hda->bnhd", cV, WV[:, t]) + muV[None, None, :, t]
+    K_rot = rope_complex(K, np.arange(n)[None, :, None], 10000.0)
+    got = O.full_decode(q, K_rot, V, lens, qpos, 0.25, 10000.0)
+    ref = O.lla_decode(q, cK, cV, muK, WK, muV, WV, t, lens, qpos, 0.25, 10000.0)
+    assert np.abs(got - ref).max() < 1e-12
+    for b in range(B):
+        for h in range(H):
+            r = sdpa(rope_complex(q[b, h], float(qpos[b]), 10000.0), K_rot[b, :lens[b], h], V[b, :lens[b], h], 0.25)
+            assert np.abs(got[b, h] - r).max() < 1e-12
+
+
 def test_softmax_special_cases():
     d, n = 8, 12
     V = syn.gaussian("pin/sm/V", (n, d))
