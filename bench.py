@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling runs)")
-    ap.add_argument("--mode", choices=["decode", "encode"], default="decode",
+    ap.add_argument("--mode", choices=["decode", "encode", "full"], default="decode",
                     help="encode: time prefill encoding of teacher stacks instead of the decode step")
     ap.add_argument("--encode-tokens", type=int, default=4096, help="tokens per encode call (encode mode)")
     ap.add_argument("--paged", action="store_true",
@@ -476,6 +476,8 @@ def main():
         a.workload += "[" + ",".join(k for k, on in (("paged", a.paged), ("self-slot", a.self_slot)) if on) + "]"
     if a.impl == "reference":
         return run_reference(a, cfg)
+    if a.mode == "full":
+        return run_full(a, cfg)
     if a.mode == "encode":
         return run_encode(a, cfg)
     return run_ours(a, cfg)
@@ -531,6 +533,73 @@ def run_encode(a, cfg):
                          "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": in_bytes}}
     print(json.dumps(line), flush=True)
     codec.close()
+    return 0
+
+
+def run_full(a, cfg):
+    """The full-cache comparator: the same decode step (T*D calls, loop-major) over an
+    uncompressed bf16 K/V cache [B][D][T][H][N+1][d] with keys stored rotated, where it fits.
+    Reports the same ctx-tokens/s and the HBM rate on the bytes the call must read
+    (its loop's keys and values)."""
+    import torch
+
+    import decode_attention_lla_b200 as lla
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    T, D, H, d = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"]
+    B, N = cfg["batch"], cfg["context"]
+    cap = N + 1
+    elems = B * D * T * cap * H * d
+    free = torch.cuda.mem_get_info(dev)[0]
+    if d != 128 or 2 * elems * 2 > free - (4 << 30):
+        print(json.dumps({"metric": "full-cache decode comparator", "unavailable":
+                          f"full K/V cache of {2 * elems * 2 / 1e9:.0f} GB does not fit (or d_head != 128)"}))
+        return 0
+    tag = f"bench/{a.workload}/full"
+    K = torch.empty(elems, dtype=torch.bfloat16, device=dev)
+    V = torch.empty(elems, dtype=torch.bfloat16, device=dev)
+    syn.fill_gaussian_bf16_(K, tag + "/K")
+    syn.fill_gaussian_bf16_(V, tag + "/V")
+    q_all = torch.empty(T, D, B, H, d, dtype=torch.float32, device=dev)
+    q_all.normal_(generator=syn.torch_generator(tag + "/q", dev))
+    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    out = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(lla.full_decode_workspace_bytes(H, d, B), dtype=torch.uint8, device=dev)
+    seq_stride = D * T * cap * H * d
+    scale = 1.0 / math.sqrt(d)
+
+    def step():
+        for t in range(T):
+            for layer in range(D):
+                off = 2 * (layer * T + t) * cap * H * d
+                lla.full_decode_attn(H, d, cfg["rope_base"], K.data_ptr() + off, V.data_ptr() + off, seq_stride, B,
+                                     cap, q_all[t, layer], lens, lens, scale, out, ws)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        e0.record()
+        for _ in range(a.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.steps
+    per_call = B * N * H * d * 2 * 2
+    peak, kind = measured_peak()
+    achieved = per_call * T * D / (ms / 1e3) / 1e9
+    line = {"metric": "full-cache decode comparator: ctx-tokens/s/GPU", "value": B * N * T * D / (ms / 1e3),
+            "unit": "ctx-tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(config_json(cfg, a.workload, 1),
+                           step=f"{T}x{D} decode calls over a full bf16 K/V cache (comparator, no LLA)"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "kernel": "full-cache decode (prologue + decode + combine, per step)",
+                         "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": per_call},
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
     return 0
 
 

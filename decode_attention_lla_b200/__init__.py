@@ -74,13 +74,17 @@ _paged_bytes = _sig("lla_paged_store_bytes", _sz, [ctypes.POINTER(CodecDesc), _i
 _encode_paged = _sig("lla_encode_paged", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _vp])
 _decode_paged = _sig("lla_decode_attn_paged", _i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f,
                                                    _vp, _vp, _sz, ctypes.POINTER(DecodeOpts), _vp])
+_full_ws = _sig("lla_full_decode_workspace_bytes", _sz, [_i, _i, _i])
+_full_decode = _sig("lla_full_decode_attn", _i, [_i, _i, _f, _vp, _vp, ctypes.c_longlong, _i, _i, _vp, _vp, _vp, _f,
+                                                 _vp, _vp, _sz, _i, _vp])
 _decode_self = _sig("lla_decode_attn_self", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _sz,
                                                  ctypes.POINTER(DecodeOpts), _vp])
 
 EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy_codec", "lla_codec_get_desc",
             "lla_store_bytes", "lla_encode", "lla_decode_workspace_bytes", "lla_decode_attn",
             "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc",
-            "lla_decode_attn_self", "lla_paged_store_bytes", "lla_encode_paged", "lla_decode_attn_paged"]
+            "lla_decode_attn_self", "lla_paged_store_bytes", "lla_encode_paged", "lla_decode_attn_paged",
+            "lla_full_decode_workspace_bytes", "lla_full_decode_attn"]
 PAGE_TOKENS = 128
 FLAG_PAGE_INVALID = 4
 
@@ -272,6 +276,20 @@ def decode_attn_paged(codec, pool, num_pages, block_table, max_pages, batch, lay
                        _ptr(q_pos), _ptr(seq_lens), _ptr(k_self), _ptr(v_self), float(scale), _ptr(out),
                        _ptr(workspace), int(workspace_bytes), ctypes.byref(opts), _stream(stream))
     _check(st, "lla_decode_attn_paged")
+
+
+def full_decode_workspace_bytes(H: int, d_head: int, batch: int) -> int:
+    return int(_full_ws(H, d_head, batch))
+
+
+def full_decode_attn(H, d_head, rope_base, k_cache, v_cache, seq_stride, batch, max_tokens, q, q_pos, seq_lens, scale,
+                     out, workspace, workspace_bytes=None, num_ctas=0, stream=None):
+    """lla_full_decode_attn: the full-cache comparator (keys cached rotated; d_head 128)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(_full_decode(H, d_head, float(rope_base), _ptr(k_cache), _ptr(v_cache), int(seq_stride), batch, max_tokens,
+                        _ptr(q), _ptr(q_pos), _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
+                        int(workspace_bytes), num_ctas, _stream(stream)), "lla_full_decode_attn")
 
 
 def raw_decode_status(fn_name, *args) -> int:

@@ -358,6 +358,36 @@ lla_status lla_decode_attn_paged(const lla_codec* c, const uint16_t* pool, int n
                          scale, out, workspace, workspace_bytes, opts, stream, k_self, v_self, smap);
 }
 
+size_t lla_full_decode_workspace_bytes(int H, int d_head, int batch) {
+    if (H < 1 || d_head != 128 || batch < 0) return 0;
+    return lla_full_workspace_bytes(H, batch);
+}
+
+lla_status lla_full_decode_attn(int H, int d_head, float rope_base, const uint16_t* k_cache, const uint16_t* v_cache,
+                                long long seq_stride, int batch, int max_tokens, const float* q,
+                                const int32_t* q_pos, const int32_t* seq_lens, float scale, float* out,
+                                void* workspace, size_t workspace_bytes, int num_ctas, void* stream) {
+    if (H < 1 || batch < 0 || max_tokens < 0 || num_ctas < 0 || !isfinite(scale) || !(rope_base > 0.f))
+        return LLA_ERR_INVALID_ARG;
+    if (d_head != 128) return LLA_ERR_UNSUPPORTED_SHAPE;
+    if (batch == 0) return LLA_OK;
+    if (!k_cache || !v_cache || !q || !q_pos || !seq_lens || !out) return LLA_ERR_INVALID_ARG;
+    if (!workspace) return LLA_ERR_WORKSPACE;
+    if (seq_stride < (long long)max_tokens * H * d_head || seq_stride % 8 != 0) return LLA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out) || !aligned16(workspace) ||
+        !aligned4(q_pos) || !aligned4(seq_lens))
+        return LLA_ERR_ALIGNMENT;
+    if (workspace_bytes < lla_full_workspace_bytes(H, batch)) return LLA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (max_tokens == 0) {
+        LLA_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(lla_ws_header), st));
+        LLA_CUDA_TRY(cudaMemsetAsync(out, 0, size_t(batch) * H * d_head * 4, st));
+        return LLA_OK;
+    }
+    return lla_full_decode(H, rope_base, k_cache, v_cache, seq_stride, batch, max_tokens, q, q_pos, seq_lens, scale,
+                           out, workspace, workspace_bytes, num_ctas, st);
+}
+
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {
     if (!workspace || !flags) return LLA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

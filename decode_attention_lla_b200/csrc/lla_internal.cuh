@@ -134,6 +134,11 @@ lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer
                          cudaStream_t stream, const lla_store_map& smap);
 
 int lla_num_sms();
+size_t lla_full_workspace_bytes(int H, int batch);
+lla_status lla_full_decode(int H, float rope_base, const uint16_t* k_cache, const uint16_t* v_cache,
+                           long long seq_stride, int batch, int max_tokens, const float* q, const int32_t* q_pos,
+                           const int32_t* seq_lens, float scale, float* out, void* workspace, size_t workspace_bytes,
+                           int num_ctas, cudaStream_t stream);
 
 #define LLA_CUDA_TRY(expr)                                   \
     do {                                                     \

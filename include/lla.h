@@ -249,6 +249,30 @@ lla_status lla_decode_attn_paged(const lla_codec* codec, const uint16_t* pool, i
                                  const lla_decode_opts* opts, void* stream);
 
 /*
+ * Comparator: decode attention over a full (uncompressed) K/V cache, the
+ * "fast path" that keeps every cached token's loop-t key and value themselves
+ * [LLA summary, "Serving Capacity"; LLA §3, "Teacher cache"].  Not part of
+ * LLA; it is here so that both paths can be timed on the same GPU where the
+ * full cache fits.
+ *   s_j = softmax_scale * <RoPE_{q_pos}(q_bh), k_bhj>,  out_bh = sum_j softmax(s)_j v_bhj
+ *   with keys cached already rotated at their positions (zero when n == 0).
+ *   k_cache, v_cache  device bf16, head-major: sequence b's head h, token j at
+ *             element b * seq_stride + (h * max_tokens + j) * d_head (seq_stride >=
+ *             H*max_tokens*d_head, a multiple of 8: a slice of a larger
+ *             [batch][layers][loops][...] cache)
+ *   q, q_pos, seq_lens, out, workspace  as lla_decode_attn (no codec: H, d_head
+ *             and rope_base are given); d_head must be 128.
+ *   num_ctas  0 = one persistent CTA per SM; otherwise that many.
+ */
+size_t lla_full_decode_workspace_bytes(int H, int d_head, int batch);
+lla_status lla_full_decode_attn(int H, int d_head, float rope_base, const uint16_t* k_cache,
+                                const uint16_t* v_cache, long long seq_stride, int batch,
+                                int max_tokens, const float* q, const int32_t* q_pos,
+                                const int32_t* seq_lens, float softmax_scale, float* out,
+                                void* workspace, size_t workspace_bytes, int num_ctas,
+                                void* stream);
+
+/*
  * lla_decode_attn_self — decode attention with the current token as a self slot
  *   [LLA §3 eq. (2)-(3)]: a token's latent is written only after its last loop
  *   (eq. (2) encodes the whole loop stack), so while it is being decoded its
