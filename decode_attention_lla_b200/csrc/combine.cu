@@ -14,17 +14,25 @@
 //   out = (sum_s w_s acc_s) W^V_up,t^T + (1 - w_self) mu^V_t + w_self v_self,
 // since the cached tokens then carry 1 - w_self of the probability.
 //
-// One CTA per (head, 16 sequences), one warp per sequence: W^V_up,t of the head
-// is staged in shared memory once, transposed so that the lanes of a warp (one
-// output dimension each) read consecutive words.
+// One CTA per (head, 8 sequences, slice of output dimensions), one warp per sequence: the rows
+// of W^V_up,t of its slice are staged in shared memory, read from global memory in their own
+// order (coalesced) and kept row-major with an odd row pitch, so that the lanes of a warp (one
+// output dimension each at a time) read distinct banks.  Small batches split d into 32-row
+// slices to fill the machine, and every CTA of a (head, sequence) then merges the records
+// itself (cheap next to the projection); large batches keep all d rows in one CTA.
 #include <math.h>
 
 #include "lla_internal.cuh"
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kSeqPerCta = kThreads / 32;  // one warp per sequence
+constexpr int kMaxRowsPerLane = 8;         // output dimensions per lane and pass
+constexpr int kAC = 8;                     // latent dims per lane held in registers while merging
+
+// Row pitch of the staged W^V_up,t: odd, so rows i and i + 1 start in different banks.
+__host__ __device__ inline int w_pitch(int rv) { return rv | 1; }
 
 struct CombineParams {
     const float* partials;
@@ -101,16 +109,17 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
     return r;
 }
 
-// One warp per (sequence, head); the CTA's sixteen warps share W^V_up,t of one head.
-__global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
+// One warp per (sequence, head); the CTA's eight warps share 32 rows of W^V_up,t of one head.
+__global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
     const int h = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y * kSeqPerCta + warp;
-    const int d = p.d, rv = p.r_v;
+    const int d = p.d, rv = p.r_v, pitch = w_pitch(rv);
+    const int rows = d / gridDim.z;  // output dimensions of this CTA's slice (gridDim.z divides d)
+    const int i0 = blockIdx.z * rows;
     extern __shared__ float smem[];
-    float* Wt = smem;                     // [rv][d]
-    float* mu = Wt + rv * d;              // [d]
-    float* abar = mu + d + warp * rv;     // [kSeqPerCta][rv]
+    float* Ws = smem;                         // [rows][pitch]: row r holds W^V_up,t[i0 + r][0..rv)
+    float* abar = Ws + rows * pitch + warp * rv;  // [kSeqPerCta][rv]
 
     size_t w_off, mu_off;
     if (p.variant == 0) {
@@ -120,12 +129,27 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
         w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(d) * rv;
         mu_off = size_t(p.layer) * p.T * p.H * d + (size_t(p.loop) * p.H + h) * d;
     }
-    // transposed into shared memory: consecutive threads write consecutive i (no bank conflicts)
-    for (int idx = threadIdx.x; idx < d * rv; idx += blockDim.x) {
-        const int a = idx / d, i = idx - a * d;
-        Wt[idx] = __ldg(p.w_up_v + w_off + size_t(i) * rv + a);
+    const float* wg = p.w_up_v + w_off + size_t(i0) * rv;
+    const int nw = rows * rv;
+    if ((rv & 3) == 0 && (reinterpret_cast<uintptr_t>(wg) & 15) == 0) {
+        // four consecutive elements of one row per load (rv % 4 == 0: no load spans two rows)
+#pragma unroll 4
+        for (int e = 4 * threadIdx.x; e < nw; e += 4 * kThreads) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(wg + e));
+            const int r = e / rv, a = e - r * rv;
+            float* w = Ws + size_t(r) * pitch + a;
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
+        }
+    } else {
+#pragma unroll 4
+        for (int e = threadIdx.x; e < nw; e += kThreads) {
+            const int r = e / rv, a = e - r * rv;
+            Ws[size_t(r) * pitch + a] = __ldg(wg + e);
+        }
     }
-    for (int i = threadIdx.x; i < d; i += blockDim.x) mu[i] = __ldg(p.mu_v + mu_off + i);
     __syncthreads();
     if (b >= p.B) return;
 
@@ -163,37 +187,61 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     L += e_self;
     float* o = p.out + bh * d;
     if (!(L > 0.f)) {  // empty context
-        for (int i = lane; i < d; i += 32) o[i] = 0.f;
+        for (int r = lane; r < rows; r += 32) o[i0 + r] = 0.f;
         return;
     }
     const float w_self = e_self / L;
-    // record weights exp(m_s - M) / L, one per lane, broadcast by shuffle
+    // abar = sum_s w_s acc_s with w_s = exp(m_s - M) / L; record weights one per lane, broadcast
+    // by shuffle; lane owns latent dims a0 + lane + 32 c, kAC of them per pass over the records
     const float invL = 1.f / L;
-    for (int a = lane; a < rv; a += 32) abar[a] = 0.f;
-    for (int sb = s0; sb < s1; sb += 32) {
-        float wgt = 0.f;
-        if (sb + lane < s1) {
-            const float* r = rec(sb + lane);
-            if (r[1] > 0.f) wgt = expf(r[0] - M) * invL;
-        }
-        const int ns = min(32, s1 - sb);
-        for (int a0 = 0; a0 < rv; a0 += 32) {  // whole warp in every iteration (shuffles)
-            const int a = a0 + lane;
-            float v = a < rv ? abar[a] : 0.f;
-#pragma unroll 4
+    for (int a0 = 0; a0 < rv; a0 += 32 * kAC) {
+        float v[kAC];
+#pragma unroll
+        for (int c = 0; c < kAC; ++c) v[c] = 0.f;
+        for (int sb = s0; sb < s1; sb += 32) {
+            float wgt = 0.f;
+            if (sb + lane < s1) {
+                const float* r = rec(sb + lane);
+                if (r[1] > 0.f) wgt = expf(r[0] - M) * invL;
+            }
+            const int ns = min(32, s1 - sb);
+#pragma unroll 2
             for (int j = 0; j < ns; ++j) {
                 const float wj = __shfl_sync(0xffffffffu, wgt, j);
-                if (wj != 0.f && a < rv) v = fmaf(rec(sb + j)[2 + a], wj, v);
+                if (wj == 0.f) continue;  // an empty record: its acc is not read
+                const float* r = rec(sb + j) + 2 + a0 + lane;
+#pragma unroll
+                for (int c = 0; c < kAC; ++c)
+                    if (a0 + lane + 32 * c < rv) v[c] = fmaf(r[32 * c], wj, v[c]);
             }
-            if (a < rv) abar[a] = v;
         }
+#pragma unroll
+        for (int c = 0; c < kAC; ++c)
+            if (a0 + lane + 32 * c < rv) abar[a0 + lane + 32 * c] = v[c];
     }
     __syncwarp();
-    // out = abar W^V_up,t^T + (1 - w_self) mu^V_t + w_self v_self
-    for (int i = lane; i < d; i += 32) {
-        float v = p.k_self ? fmaf(w_self, p.v_self[bh * d + i], (1.f - w_self) * mu[i]) : mu[i];
-        for (int a = 0; a < rv; ++a) v = fmaf(abar[a], Wt[a * d + i], v);
-        o[i] = v;
+    // out_i = abar . W^V_up,t[i] + (1 - w_self) mu^V_t[i] + w_self v_self[i] for i = i0 + r,
+    // r = r0 + lane + 32 k; the rows of a lane keep independent accumulation chains
+    for (int r0 = 0; r0 < rows; r0 += 32 * kMaxRowsPerLane) {
+        float acc[kMaxRowsPerLane];
+#pragma unroll
+        for (int k = 0; k < kMaxRowsPerLane; ++k) acc[k] = 0.f;
+        const float* wr = Ws + size_t(min(r0 + lane, rows - 1)) * pitch;
+        const int nk = min(kMaxRowsPerLane, (rows - r0 + 31) / 32);
+        for (int a = 0; a < rv; ++a) {
+            const float x = abar[a];
+#pragma unroll
+            for (int k = 0; k < kMaxRowsPerLane; ++k)
+                if (k < nk && r0 + lane + 32 * k < rows) acc[k] = fmaf(x, wr[size_t(32 * k) * pitch + a], acc[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxRowsPerLane; ++k) {
+            const int r = r0 + lane + 32 * k;
+            if (k >= nk || r >= rows) break;
+            const int i = i0 + r;
+            const float m = __ldg(p.mu_v + mu_off + i);
+            o[i] = acc[k] + (p.k_self ? fmaf(w_self, p.v_self[bh * d + i], (1.f - w_self) * m) : m);
+        }
     }
 }
 
@@ -241,9 +289,13 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     p.k_self = call.k_self;
     p.v_self = call.v_self;
     p.scale = call.scale;
-    const size_t smem = (size_t(ds.r_v) * ds.d_head + ds.d_head + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
+    // split d into 32-row slices while the grid is short of two CTAs per SM
+    const int seq_ctas = (call.batch + kSeqPerCta - 1) / kSeqPerCta;
+    int z = 1;
+    while (ds.d_head % (64 * z) == 0 && ds.H * seq_ctas * z < 2 * lla_num_sms()) z *= 2;
+    const size_t smem = (size_t(w_pitch(ds.r_v)) * (ds.d_head / z) + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    dim3 grid(ds.H, (call.batch + kSeqPerCta - 1) / kSeqPerCta);
+    dim3 grid(ds.H, seq_ctas, z);
     combine_kernel<<<grid, kThreads, smem, call.stream>>>(p);
     LLA_CUDA_TRY(cudaGetLastError());
     return LLA_OK;

@@ -689,30 +689,56 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         if (threadIdx.x == 0) p.P[p.B] = carry;
         return;
     }
-    // one warp per (sequence, head): this head's rows of the sequence's M_q image
+    // CTA (head h, SPC sequences), WPS warps per sequence (SPC * WPS = 8): this head's rows of
+    // each sequence's M_q image.  W^K_up,t of the head ([n][i], row RK = mu) is staged in shared
+    // memory once; the items of a sequence are spread over its warps so that every lane keeps
+    // its few values in registers between the max and the write.
     constexpr int DH = C::DH, RK = C::RK, half = DH / 2, KC = DH / 8;
     constexpr int NITEM = (RK + 1) * KC;  // (row, 8-wide k chunk) items
-    const int bh = (blockIdx.x - 1) * 8 + w;
-    if (bh >= p.B * C::H) return;
-    const int b = bh / C::H, h = bh - b * C::H;
-    __shared__ __align__(16) float qr_all[8][DH];
-    float* qr = qr_all[w];
+    constexpr int WPS = NITEM >= 1024 ? 8 : NITEM >= 512 ? 4 : NITEM >= 256 ? 2 : 1;
+    constexpr int SPC = 8 / WPS;
+    static_assert(DH % 4 == 0, "float4 staging");
+    extern __shared__ __align__(16) float pro_smem[];
+    __shared__ float red[8];
+    const int k = blockIdx.x - 1;
+    const int sl = w / WPS, wi = w % WPS;
+    const int h = k % C::H, b = (k / C::H) * SPC + sl;
+    const bool active = b < p.B;
     const size_t slot = p.variant == 0 ? (size_t(p.layer) * C::H + h) * p.T + p.loop
                                        : (size_t(p.layer) * p.T + p.loop) * C::H + h;
-    const float* wt = p.w_up_k_t + slot * size_t(RK + 1) * DH;  // [n][i], row RK = mu
-    int qp = p.q_pos[b];
-    if (qp < 0 || qp >= p.max_pos) {
-        qp = qp < 0 ? 0 : p.max_pos - 1;
-        if (h == 0 && lane == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
+    float* wt = pro_smem;
+    // W loads all issued up front (their latency overlaps the rotation of q below), stored after
+    constexpr int NW4 = (RK + 1) * DH / 4, WPT = (NW4 + 255) / 256;
+    float4 wreg[WPT];
+    {
+        const float4* wg = reinterpret_cast<const float4*>(p.w_up_k_t + slot * size_t(RK + 1) * DH);
+#pragma unroll
+        for (int j = 0; j < WPT; ++j) {
+            const int e = threadIdx.x + 256 * j;
+            if (e < NW4) wreg[j] = __ldg(wg + e);
+        }
     }
-    const float* qv = p.q + (size_t(b) * C::H + h) * DH;
-    for (int i = lane; i < half; i += 32) {
-        const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
-        const float lo = qv[i], hi = qv[i + half];
-        qr[i] = p.scale * (lo * c - hi * sn);
-        qr[i + half] = p.scale * (hi * c + lo * sn);
+    float* qr = pro_smem + (RK + 1) * DH + sl * DH;
+    if (active) {
+        int qp = p.q_pos[b];
+        if (qp < 0 || qp >= p.max_pos) {
+            qp = qp < 0 ? 0 : p.max_pos - 1;
+            if (h == 0 && wi == 0 && lane == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
+        }
+        const float* qv = p.q + (size_t(b) * C::H + h) * DH;
+        for (int i = wi * 32 + lane; i < half; i += WPS * 32) {
+            const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
+            const float lo = qv[i], hi = qv[i + half];
+            qr[i] = p.scale * (lo * c - hi * sn);
+            qr[i + half] = p.scale * (hi * c + lo * sn);
+        }
     }
-    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < WPT; ++j) {
+        const int e = threadIdx.x + 256 * j;
+        if (e < NW4) reinterpret_cast<float4*>(wt)[e] = wreg[j];
+    }
+    __syncthreads();
     // element (n, k): k < d/2: q'_k w_k + q'_{k+d/2} w_{k+d/2};  k >= d/2: q'_{i+d/2} w_i - q'_i w_{i+d/2}
     auto item = [&](int e, float* v) {
         const int n = e / KC, k0 = (e - n * KC) * 8;
@@ -723,7 +749,7 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         const float4* qh = reinterpret_cast<const float4*>(qr + i0 + half);
 #pragma unroll
         for (int u4 = 0; u4 < 2; ++u4) {
-            const float4 a = __ldg(wl + u4), bb = __ldg(wh + u4), x = ql[u4], y = qh[u4];
+            const float4 a = wl[u4], bb = wh[u4], x = ql[u4], y = qh[u4];
             if (k0 < half) {
                 v[4 * u4 + 0] = x.x * a.x + y.x * bb.x;
                 v[4 * u4 + 1] = x.y * a.y + y.y * bb.y;
@@ -737,16 +763,17 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
             }
         }
     };
-    // small ranks: all of this lane's values stay in registers (one pass over W);
-    // large ranks: a max pass, then the values are recomputed for the write pass
-    constexpr int NPL = (NITEM + 31) / 32;  // items per lane
+    // few items per lane: the values stay in registers (one pass over W);
+    // many: a max pass, then the values are recomputed for the write pass
+    constexpr int NPL = (NITEM + 32 * WPS - 1) / (32 * WPS);  // items per lane
     constexpr bool KEEP = NPL <= 12;
+    const int e0 = wi * 32 + lane;
     float keep[KEEP ? NPL : 1][8];
     float mx = 0.f;
 #pragma unroll
     for (int it = 0; it < NPL; ++it) {
-        const int e = lane + 32 * it;
-        if (e < NITEM) {
+        const int e = e0 + 32 * WPS * it;
+        if (active && e < NITEM) {
             float* v = keep[KEEP ? it : 0];
             item(e, v);
 #pragma unroll
@@ -755,6 +782,10 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[w] = mx;
+    __syncthreads();
+    if (!active) return;
+    for (int j = 0; j < WPS; ++j) mx = fmaxf(mx, red[sl * WPS + j]);
     // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
     int e2 = 0;
     float scale = 1.f;
@@ -766,7 +797,7 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
     uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
 #pragma unroll
     for (int it = 0; it < NPL; ++it) {
-        const int e = lane + 32 * it;
+        const int e = e0 + 32 * WPS * it;
         if (e >= NITEM) break;
         float vv[8];
         if (!KEEP) item(e, vv);
@@ -778,12 +809,12 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         for (int u = 0; u < 8; ++u) hv[u] = __float2half_rn(v[u] * scale);
         *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = *reinterpret_cast<const uint4*>(hv);
     }
-    if (hg == 0)  // the group's padding rows
+    if (hg == 0 && wi == 0)  // the group's padding rows
         for (int e = lane; e < (C::NG - C::HG * (RK + 1)) * KC; e += 32) {
             const int rowi = C::HG * (RK + 1) + e / KC, k0 = (e % KC) * 8;
             *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = make_uint4(0, 0, 0, 0);
         }
-    if (lane == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
+    if (wi == 0 && lane == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -879,7 +910,11 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.smap = call.smap;
     // split records start empty (l = 0); the combine skips them
     LLA_CUDA_TRY(cudaMemsetAsync(pp.records, 0, pp.n_record_floats * sizeof(float), call.stream));
-    tc_prologue_kernel<C><<<1 + (B * C::H + 7) / 8, 256, 0, call.stream>>>(pp);
+    constexpr int pro_items = (C::RK + 1) * (C::DH / 8);
+    constexpr int pro_spc = pro_items >= 1024 ? 1 : pro_items >= 512 ? 2 : pro_items >= 256 ? 4 : 8;  // 8 / WPS
+    const size_t pro_smem = size_t(C::RK + 1 + pro_spc) * C::DH * sizeof(float);
+    LLA_CUDA_TRY(cudaFuncSetAttribute(tc_prologue_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pro_smem)));
+    tc_prologue_kernel<C><<<1 + C::H * ((B + pro_spc - 1) / pro_spc), 256, pro_smem, call.stream>>>(pp);
     LLA_CUDA_TRY(cudaGetLastError());
 
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).  Per-head
