@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
         }
     }
     __syncthreads();
+    lla_grid_dependency_wait();  // W above is a constant; the records come from the decode kernel
     if (b >= p.B) return;
 
     const RecordSet rs = record_set(p, b, h);
@@ -296,7 +297,7 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     const size_t smem = (size_t(w_pitch(ds.r_v)) * (ds.d_head / z) + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     dim3 grid(ds.H, seq_ctas, z);
-    combine_kernel<<<grid, kThreads, smem, call.stream>>>(p);
-    LLA_CUDA_TRY(cudaGetLastError());
+    // overlapped with the decode kernel's tail, unless an event follows that kernel for timing
+    LLA_CUDA_TRY(lla_launch(combine_kernel, grid, dim3(kThreads), smem, call.stream, call.ev_end == nullptr, p));
     return LLA_OK;
 }

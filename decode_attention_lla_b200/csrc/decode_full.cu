@@ -166,6 +166,7 @@ __global__ void __maxnreg__(kMaxRegs) full_decode(const __grid_constant__ CUtens
         fence_mbar_init();
     }
     __syncthreads();
+    lla_grid_dependency_wait();  // the prologue's tile plan and q' are read from here on
 
     TileWalker wk;
     wk.init(p.P, p.B * p.H, p.G, blockIdx.x, 1);
@@ -206,7 +207,7 @@ __global__ void __maxnreg__(kMaxRegs) full_decode(const __grid_constant__ CUtens
     const int qd = cw % kQuarters;   // token rows [32 qd, 32 qd + 32) of those tiles
     float* qw = qbuf + cw * kD;  // this warp's copy of q', reloaded per stream
     float m = -INFINITY, l = 0.f;
-    float acc[4];             // dimensions 4 lane .. 4 lane + 3
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // dimensions 4 lane .. 4 lane + 3
     uint32_t n = 0;
     int prev = -1;
     bool ok = true;
@@ -307,6 +308,7 @@ __global__ void __maxnreg__(kMaxRegs) full_decode(const __grid_constant__ CUtens
 // One warp per (sequence, head): merge the records of the CTAs that covered the stream.
 __global__ void __launch_bounds__(256) full_combine(FullParams p, float* out) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    lla_grid_dependency_wait();  // the records come from the decode kernel
     const long long s = (long long)blockIdx.x * 8 + warp;
     if (s >= (long long)p.B * p.H) return;
     float4* o = reinterpret_cast<float4*>(out + s * kD) + lane;
@@ -425,9 +427,8 @@ lla_status lla_full_decode(int H, float rope_base, const uint16_t* k_cache, cons
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return LLA_ERR_CUDA;
     LLA_CUDA_TRY(cudaFuncSetAttribute(full_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
-    full_decode<<<G, kThreads, kSmem, stream>>>(kmap, vmap, p);
-    LLA_CUDA_TRY(cudaGetLastError());
-    full_combine<<<int((batch * (long long)H + 7) / 8), 256, 0, stream>>>(p, out);
-    LLA_CUDA_TRY(cudaGetLastError());
+    // each kernel is scheduled while its predecessor drains and waits for its results
+    LLA_CUDA_TRY(lla_launch(full_decode, dim3(G), dim3(kThreads), kSmem, stream, true, kmap, vmap, p));
+    LLA_CUDA_TRY(lla_launch(full_combine, dim3(int((batch * (long long)H + 7) / 8)), dim3(256), 0, stream, true, p, out));
     return LLA_OK;
 }

@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    lla_grid_dependency_wait();  // the prologue's tile plan and M_q images are read from here on
 
     TileWalker wk;
     wk.init(p.P, p.B, p.G, blockIdx.x, C::PARTS);
@@ -972,8 +973,8 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     else kernel = tc_decode_kernel<C>;
     LLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     if (call.ev_begin) LLA_CUDA_TRY(cudaEventRecord(call.ev_begin, call.stream));
-    kernel<<<G, C::THREADS, C::SMEM, call.stream>>>(maps, tp);
-    LLA_CUDA_TRY(cudaGetLastError());
+    // overlapped with the prologue's tail, unless events bracket the kernel for timing
+    LLA_CUDA_TRY(lla_launch(kernel, dim3(G), dim3(C::THREADS), C::SMEM, call.stream, call.ev_begin == nullptr, maps, tp));
     if (call.ev_end) LLA_CUDA_TRY(cudaEventRecord(call.ev_end, call.stream));
     lla_tc_ranges ranges;
     ranges.P = pp.P;

@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    lla_grid_dependency_wait();  // the prologue's tile plan and M_q images are read from here on
 
     TileWalker wk;
     wk.init(p.P, p.B, p.G, blockIdx.x, C::PARTS);

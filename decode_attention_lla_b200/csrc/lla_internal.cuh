@@ -140,6 +140,31 @@ lla_status lla_full_decode(int H, float rope_base, const uint16_t* k_cache, cons
                            const int32_t* seq_lens, float scale, float* out, void* workspace, size_t workspace_bytes,
                            int num_ctas, cudaStream_t stream);
 
+// ---- programmatic dependent launch ----------------------------------------------------------
+// The kernels of one call run back to back in a stream.  A kernel launched by lla_launch with
+// pdl = true is scheduled as the CTAs of the kernel before it exit (none of them triggers its
+// dependents early: measured slower, the dependents then take SM resources the predecessor's
+// last CTAs still need); it calls lla_grid_dependency_wait() before it touches anything that
+// kernel writes (a no-op after a plain launch), so its launch and set-up overlap that kernel's
+// tail.
+__device__ __forceinline__ void lla_grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t lla_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 #define LLA_CUDA_TRY(expr)                                   \
     do {                                                     \
         cudaError_t _e = (expr);                             \
