@@ -41,7 +41,8 @@ DEFAULT_WORKLOAD = "ouro_rho21_b768_n4096"
 # kernels the library launches per call (our own kernels only; memsets excluded)
 LAUNCHES_PER_DECODE = {"simt": 2, "tc": 3}
 LAUNCHES_PER_ENCODE = 1
-KERNEL_SOURCES = {"simt": ["decode_simt.cu", "sm100.cuh"], "tc": ["decode_tc.cu", "decode_tc2d.cuh", "sm100.cuh"]}
+KERNEL_SOURCES = {"simt": ["decode_simt.cu", "sm100.cuh"], "tc": ["decode_tc.cu", "decode_tc2d.cuh", "sm100.cuh", "walk.cuh"],
+                  "full": ["decode_full.cu", "sm100.cuh", "walk.cuh"]}
 
 
 def parse():
@@ -596,7 +597,8 @@ def run_full(a, cfg):
             "config": dict(config_json(cfg, a.workload, 1),
                            step=f"{T}x{D} decode calls over a full bf16 K/V cache (comparator, no LLA)"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": None, "kernel": "full-cache decode (prologue + decode + combine, per step)",
+                         "traffic": traffic_record("full", a.workload),
+                         "kernel": "full-cache decode (prologue + decode + combine, per step)",
                          "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": per_call},
             "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
