@@ -65,6 +65,9 @@ def parse():
                     help="latent store as a pool of 128-token pages in shuffled order with a block table")
     ap.add_argument("--self-slot", action="store_true",
                     help="decode calls attend to the current token's exact K/V as well (lla_decode_attn_self)")
+    ap.add_argument("--final-loop", action="store_true",
+                    help="full mode: cache only the final loop's K/V and use it for every loop (zero-parameter "
+                         "matched-budget baseline: 1/T of the full cache)")
     return ap.parse_args()
 
 
@@ -540,8 +543,9 @@ def run_encode(a, cfg):
 def run_full(a, cfg):
     """The full-cache comparator: the same decode step (T*D calls, loop-major) over an
     uncompressed bf16 K/V cache [B][D][T][H][N+1][d] with keys stored rotated, where it fits.
-    Reports the same ctx-tokens/s and the HBM rate on the bytes the call must read
-    (its loop's keys and values)."""
+    With --final-loop the cache keeps one loop slot per layer ([B][D][1][H][N+1][d], the final
+    loop's K/V) and every loop's call reads it.  Reports the same ctx-tokens/s and the HBM rate
+    on the bytes the call must read (one loop's keys and values)."""
     import torch
 
     import decode_attention_lla_b200 as lla
@@ -551,7 +555,8 @@ def run_full(a, cfg):
     T, D, H, d = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"]
     B, N = cfg["batch"], cfg["context"]
     cap = N + 1
-    elems = B * D * T * cap * H * d
+    TS = 1 if a.final_loop else T  # loop slots kept per layer
+    elems = B * D * TS * cap * H * d
     free = torch.cuda.mem_get_info(dev)[0]
     if d != 128 or 2 * elems * 2 > free - (4 << 30):
         print(json.dumps({"metric": "full-cache decode comparator", "unavailable":
@@ -567,13 +572,13 @@ def run_full(a, cfg):
     lens = torch.full((B,), N, dtype=torch.int32, device=dev)
     out = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     ws = torch.empty(lla.full_decode_workspace_bytes(H, d, B), dtype=torch.uint8, device=dev)
-    seq_stride = D * T * cap * H * d
+    seq_stride = D * TS * cap * H * d
     scale = 1.0 / math.sqrt(d)
 
     def step():
         for t in range(T):
             for layer in range(D):
-                off = 2 * (layer * T + t) * cap * H * d
+                off = 2 * (layer * TS + (0 if a.final_loop else t)) * cap * H * d
                 lla.full_decode_attn(H, d, cfg["rope_base"], K.data_ptr() + off, V.data_ptr() + off, seq_stride, B,
                                      cap, q_all[t, layer], lens, lens, scale, out, ws)
 
@@ -591,11 +596,13 @@ def run_full(a, cfg):
     per_call = B * N * H * d * 2 * 2
     peak, kind = measured_peak()
     achieved = per_call * T * D / (ms / 1e3) / 1e9
-    line = {"metric": "full-cache decode comparator: ctx-tokens/s/GPU", "value": B * N * T * D / (ms / 1e3),
+    what = "final-loop reuse (one loop slot per layer)" if a.final_loop else "full-cache decode comparator"
+    line = {"metric": f"{what}: ctx-tokens/s/GPU", "value": B * N * T * D / (ms / 1e3),
             "unit": "ctx-tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(config_json(cfg, a.workload, 1),
-                           step=f"{T}x{D} decode calls over a full bf16 K/V cache (comparator, no LLA)"),
+                           step=f"{T}x{D} decode calls over a full bf16 K/V cache (comparator, no LLA)",
+                           cache_gb=2 * elems * 2 / 1e9, loop_slots=TS),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic_record("full", a.workload),
                          "kernel": "full-cache decode (prologue + decode + combine, per step)",

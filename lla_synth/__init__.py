@@ -35,6 +35,11 @@ CONFIGS = {
     "huginn_t32_b16_n32768": dict(D=4, T=32, H=16, d_head=128, r_k=96, r_v=160, variant=0, batch=16,
                                   context=32768, rope_base=10000.0, traj_rank=24, noise_var=1e-2,
                                   mu_var=0.1),
+    # matched-axis baseline at the ratio-21.3 cache budget: per-loop MLA, a latent over the head
+    # axis of each (layer, loop) with no sharing across loops.  The 24 layers x 4 loops become 96
+    # single-loop slots; 4 loops x 192 elements = 16 heads x 48 elements per token and layer.
+    "mla_perloop_b768_n4096": dict(D=96, T=1, H=16, d_head=128, r_k=64, r_v=128, variant=1, batch=768,
+                                   context=4096, rope_base=10000.0, mu_var=0.1),
 }
 
 

@@ -164,9 +164,11 @@ def test_split_count_invariance(impl, ctas, ci):
 @pytest.mark.parametrize("c", [dict(D=2, T=2, H=4, d_head=16, r_k=12, r_v=20, B=3, N=200, lens=[200, 0, 77]),
                                dict(D=1, T=4, H=16, d_head=128, r_k=64, r_v=128, B=2, N=300, lens=[300, 130]),
                                dict(D=2, T=4, H=16, d_head=128, r_k=64, r_v=128, B=5, N=900,
-                                    lens=[900, 0, 1, 385, 640])])
+                                    lens=[900, 0, 1, 385, 640]),
+                               # T = 1: per-loop MLA, the head-axis latent of one loop
+                               dict(D=3, T=1, H=16, d_head=128, r_k=64, r_v=128, B=3, N=400, lens=[400, 5, 256])])
 def test_2d_matches_oracle(c):
-    tag = f"2d/{c['d_head']}"
+    tag = f"2d/{c['d_head']}/{c['T']}"
     cfg = dict(c, variant=1, rope_base=10000.0, mu_var=0.1)
     codec = rounded_codec(syn.seeded_codec(cfg, tag))
     B, N, D = c["B"], c["N"], c["D"]

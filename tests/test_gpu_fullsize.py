@@ -65,9 +65,14 @@ def test_full_size_sampled(name, layer, loop, sample):
     torch.cuda.empty_cache()
 
 
-def test_full_size_2d_sampled():
-    """LLA-2D at batch 256 x 8192 (19.3 GB store), one layer filled, sampled sequences."""
-    name, layer, loop, sample = "ouro_2d_b256_n8192", 11, 2, [0, 1, 128, 255]
+@pytest.mark.parametrize("name,layer,loop,sample", [
+    ("ouro_2d_b256_n8192", 11, 2, [0, 1, 128, 255]),
+    # per-loop MLA at the ratio-21.3 budget: 96 single-loop slots, 116 GB store
+    ("mla_perloop_b768_n4096", 57, 0, [0, 300, 767]),
+])
+def test_full_size_2d_sampled(name, layer, loop, sample):
+    """LLA-2D (batch 256 x 8192, 19.3 GB store) and per-loop MLA (T = 1, batch 768 x 4096), one
+    layer slot filled, sampled sequences."""
     cfg = syn.CONFIGS[name]
     D, T, H, d, rk, rv = cfg["D"], cfg["T"], cfg["H"], cfg["d_head"], cfg["r_k"], cfg["r_v"]
     B, N = cfg["batch"], cfg["context"]
