@@ -58,13 +58,14 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling runs)")
-    ap.add_argument("--mode", choices=["decode", "encode", "full"], default="decode",
+    ap.add_argument("--mode", choices=["decode", "encode", "full", "fit"], default="decode",
                     help="encode: time prefill encoding of teacher stacks instead of the decode step")
     ap.add_argument("--encode-tokens", type=int, default=4096, help="tokens per encode call (encode mode)")
     ap.add_argument("--paged", action="store_true",
                     help="latent store as a pool of 128-token pages in shuffled order with a block table")
     ap.add_argument("--self-slot", action="store_true",
                     help="decode calls attend to the current token's exact K/V as well (lla_decode_attn_self)")
+    ap.add_argument("--calib", type=int, default=1024, help="fit mode: calibration stacks per (layer, head, axis)")
     ap.add_argument("--final-loop", action="store_true",
                     help="full mode: cache only the final loop's K/V and use it for every loop (zero-parameter "
                          "matched-budget baseline: 1/T of the full cache)")
@@ -484,7 +485,96 @@ def main():
         return run_full(a, cfg)
     if a.mode == "encode":
         return run_encode(a, cfg)
+    if a.mode == "fit":
+        return run_fit(a, cfg)
     return run_ours(a, cfg)
+
+
+# fp64 CUDA-core peak: 148 SMs x 64 fp64 FMA per clock x 2 flop at the 1965 MHz maximum SM clock
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+
+
+def run_fit(a, cfg):
+    """GPU codec fit (lla_fit_codec): the SVD initialisation of every (layer, head) codec of the
+    workload, K and V axes, from `--calib` seeded calibration stacks each (S = T*d_head, or
+    T*H*d_head for 2D).  A step fits all of them; reports codec fits per second.  The CPU
+    baseline is the oracle's FP64 SVD fit on a bounded sample of the same problems."""
+    import torch
+
+    import decode_attention_lla_b200 as lla
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    T, D, H, d = cfg["T"], cfg["D"], cfg["H"], cfg["d_head"]
+    two_d = cfg.get("variant", 0) == 1
+    S = T * d * (H if two_d else 1)
+    P = D * (1 if two_d else H)  # problems per axis
+    n = a.calib
+    R = cfg.get("traj_rank", 24)
+    noise = cfg.get("noise_var", 1e-2)
+    tag = f"bench/{a.workload}/fit"
+    # calibration stacks: a few distinct seeded slots repeated over the problems (the fit's cost
+    # does not depend on the values)
+    base = np.stack([syn.smooth_stacks(f"{tag}/{i}", n, T, d * (H if two_d else 1), R, noise,
+                                       syn.gaussian(f"{tag}/mu/{i}", S, cfg.get("mu_var", 0.1)))
+                     for i in range(4)]).astype(np.float32)
+    Xh = np.concatenate([base] * ((P + 3) // 4))[:P]
+    X = torch.from_numpy(Xh).to(dev)
+    out = {}
+    for axis, r in (("k", cfg["r_k"]), ("v", cfg["r_v"])):
+        ws = torch.empty(lla.fit_codec_workspace_bytes(P, n, S, r), dtype=torch.uint8, device=dev)
+        out[axis] = (r, ws, torch.empty(P, S, device=dev), torch.empty(P, S, r, device=dev),
+                     torch.empty(P, r, device=dev))
+
+    def step():
+        for axis in ("k", "v"):
+            r, ws, mu, W, sig = out[axis]
+            lla.fit_codec(P, n, S, r, X, mu, W, sig, ws)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        e0.record()
+        for _ in range(a.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.steps
+    flags = max(lla.workspace_flags(out[ax][1]) for ax in ("k", "v"))
+    # fp64 GEMM work of the algorithm (Gram, 24 products with G, 13 shifted CholeskyQR3, Ritz)
+    def gemm_flops(r):
+        m = min(n, S)
+        k = min(m, max(2 * r, r + 16))
+        orths = 1 + 12
+        back = 2.0 * S * n * r if n < S else 0.0  # left singular vectors -> right ones
+        return P * (2.0 * n * S * m / 2 + 24 * 2.0 * m * m * k + orths * 3 * 2 * 2.0 * m * k * k
+                    + 2.0 * m * m * k + 2.0 * m * k * k + 2.0 * m * k * r + back)
+    fl = gemm_flops(cfg["r_k"]) + gemm_flops(cfg["r_v"])
+    achieved = fl / (ms / 1e3) / 1e12
+    # CPU baseline: the oracle's FP64 fit on a bounded sample of the same problems
+    from oracle import lla_oracle as O
+    t0, done, cores = time.perf_counter(), 0, os.cpu_count()
+    while time.perf_counter() - t0 < a.cpu_seconds / 2 and done < 2 * P:
+        axis_r = cfg["r_k"] if done % 2 == 0 else cfg["r_v"]
+        O.fit_codec_svd(Xh[done % P].astype(np.float64), axis_r)
+        done += 1
+    cpu_rate = done / (time.perf_counter() - t0)
+    line = {"metric": "GPU codec fit: (layer, head, axis) codecs fitted per second", "value": 2 * P / (ms / 1e3),
+            "unit": "codec fits/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": a.workload, "problems_per_axis": P, "calib_stacks": n, "S": S,
+                       "r_k": cfg["r_k"], "r_v": cfg["r_v"], "iterations": 24, "flags": flags},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP64_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": achieved / FP64_PEAK_TFLOPS, "traffic": None,
+                         "kernel": "whole fit (fp64 GEMM work / fit time; latency of the small factorisations bounds it)",
+                         "peak_source": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x 1.965 GHz"},
+            "cpu_baseline": {"value": cpu_rate, "unit": "codec fits/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{done} FP64 SVD fits of {n} x {S} stacks"},
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_encode(a, cfg):

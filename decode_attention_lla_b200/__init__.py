@@ -77,6 +77,8 @@ _decode_paged = _sig("lla_decode_attn_paged", _i, [_vp, _vp, _i, _vp, _i, _i, _i
 _full_ws = _sig("lla_full_decode_workspace_bytes", _sz, [_i, _i, _i])
 _full_decode = _sig("lla_full_decode_attn", _i, [_i, _i, _f, _vp, _vp, ctypes.c_longlong, _i, _i, _vp, _vp, _vp, _f,
                                                  _vp, _vp, _sz, _i, _vp])
+_fit_ws = _sig("lla_fit_codec_workspace_bytes", _sz, [_i, _i, _i, _i])
+_fit = _sig("lla_fit_codec", _i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp])
 _decode_self = _sig("lla_decode_attn_self", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _sz,
                                                  ctypes.POINTER(DecodeOpts), _vp])
 
@@ -84,9 +86,11 @@ EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy
             "lla_store_bytes", "lla_encode", "lla_decode_workspace_bytes", "lla_decode_attn",
             "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc",
             "lla_decode_attn_self", "lla_paged_store_bytes", "lla_encode_paged", "lla_decode_attn_paged",
-            "lla_full_decode_workspace_bytes", "lla_full_decode_attn"]
+            "lla_full_decode_workspace_bytes", "lla_full_decode_attn", "lla_fit_codec_workspace_bytes",
+            "lla_fit_codec"]
 PAGE_TOKENS = 128
 FLAG_PAGE_INVALID = 4
+FLAG_FIT_BREAKDOWN = 8
 
 
 class LLAError(RuntimeError):
@@ -290,6 +294,19 @@ def full_decode_attn(H, d_head, rope_base, k_cache, v_cache, seq_stride, batch, 
     _check(_full_decode(H, d_head, float(rope_base), _ptr(k_cache), _ptr(v_cache), int(seq_stride), batch, max_tokens,
                         _ptr(q), _ptr(q_pos), _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
                         int(workspace_bytes), num_ctas, _stream(stream)), "lla_full_decode_attn")
+
+
+def fit_codec_workspace_bytes(problems: int, n: int, S: int, r: int) -> int:
+    return int(_fit_ws(problems, n, S, r))
+
+
+def fit_codec(problems, n, S, r, X, mu, w_down, sigma, workspace, iters=0, workspace_bytes=None, stream=None):
+    """lla_fit_codec: mu, W_down (top-r right singular vectors of the centred stacks) and the top
+    singular values of `problems` calibration sets X [problems][n][S] (device float32)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(_fit(problems, n, S, r, _ptr(X), _ptr(mu), _ptr(w_down), _ptr(sigma) if sigma is not None else None,
+                iters, _ptr(workspace), int(workspace_bytes), _stream(stream)), "lla_fit_codec")
 
 
 def raw_decode_status(fn_name, *args) -> int:

@@ -388,6 +388,29 @@ lla_status lla_full_decode_attn(int H, int d_head, float rope_base, const uint16
                            out, workspace, workspace_bytes, num_ctas, st);
 }
 
+size_t lla_fit_codec_workspace_bytes(int problems, int n, int S, int r) {
+    if (problems < 1 || n < 1 || S < 1 || r < 1 || r > (n < S ? n : S) || (n < S ? n : S) > 32768 ||
+        !lla_fit_shape_ok(n, S, r))
+        return 0;
+    return lla_fit_workspace_bytes_impl(problems, n, S, r);
+}
+
+lla_status lla_fit_codec(int problems, int n, int S, int r, const float* X, float* mu, float* w_down, float* sigma,
+                         int iters, void* workspace, size_t workspace_bytes, void* stream) {
+    if (problems < 0 || n < 1 || S < 1 || r < 1 || iters < 0) return LLA_ERR_INVALID_ARG;
+    const int m = n < S ? n : S;
+    if (r > m) return LLA_ERR_INVALID_ARG;
+    if (m > 32768 || !lla_fit_shape_ok(n, S, r)) return LLA_ERR_UNSUPPORTED_SHAPE;
+    if (problems == 0) return LLA_OK;
+    if (!X || !mu || !w_down) return LLA_ERR_INVALID_ARG;
+    if (!workspace) return LLA_ERR_WORKSPACE;
+    if (!aligned4(X) || !aligned4(mu) || !aligned4(w_down) || (sigma && !aligned4(sigma)) || !aligned16(workspace))
+        return LLA_ERR_ALIGNMENT;
+    if (workspace_bytes < lla_fit_workspace_bytes_impl(problems, n, S, r)) return LLA_ERR_WORKSPACE;
+    return lla_fit(problems, n, S, r, X, mu, w_down, sigma, iters == 0 ? 24 : iters, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {
     if (!workspace || !flags) return LLA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -47,6 +47,7 @@ enum : uint32_t {
     LLA_FLAG_SEQ_LEN_CLAMPED = 1u,
     LLA_FLAG_POS_CLAMPED = 2u,
     LLA_FLAG_PAGE_INVALID = 4u,
+    LLA_FLAG_FIT_BREAKDOWN = 8u,  // codec fit: a Cholesky pivot was not positive
 };
 
 // Where the rows of a latent store live.  Contiguous: [batch][D][max_tokens][row].  Paged: a
@@ -134,6 +135,10 @@ lla_status lla_encode_tc(const lla_codec* c, const uint16_t* x, int n, int layer
                          cudaStream_t stream, const lla_store_map& smap);
 
 int lla_num_sms();
+size_t lla_fit_workspace_bytes_impl(int P, int n, int S, int r);
+bool lla_fit_shape_ok(int n, int S, int r);
+lla_status lla_fit(int P, int n, int S, int r, const float* X, float* mu_out, float* w_out, float* sig_out, int iters,
+                   void* workspace, cudaStream_t stream);
 size_t lla_full_workspace_bytes(int H, int batch);
 lla_status lla_full_decode(int H, float rope_base, const uint16_t* k_cache, const uint16_t* v_cache,
                            long long seq_stride, int batch, int max_tokens, const float* q, const int32_t* q_pos,

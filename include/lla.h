@@ -299,6 +299,37 @@ lla_status lla_decode_attn_self(const lla_codec* codec, const uint16_t* store, i
                                 void* stream);
 
 /*
+ * Codec fit on the GPU — the SVD initialisation of W_down [LLA §3,
+ * "Initialisation and conversion"]: for each of `problems` independent
+ * (layer, head, axis) slots, the calibration stacks X (n x S; S = T*d_head,
+ * or T*H*d_head for the 2D variant) are centred with their mean and W_down is
+ * the top-r right singular vectors of X - mu, each column flipped so that its
+ * entry of largest magnitude is positive.  The loop-t up-projection is then
+ * the loop-t row slice of W_down, and mu_t the loop-t slice of mu.
+ *   Computed in fp64: the Gram matrix of the smaller side, subspace iteration
+ *   with a block of min(n, S, max(2r, r+16)) columns orthonormalised by shifted
+ *   CholeskyQR3, then Rayleigh-Ritz with cyclic Jacobi rotations.  The
+ *   singular values and the fitted subspace converge with the iteration count
+ *   (24 by default; ~1e-8 relative on smooth low-rank-plus-noise stacks).
+ *   X        device float32 [problems][n][S]
+ *   mu       device float32 [problems][S] (out)
+ *   w_down   device float32 [problems][S][r] (out)
+ *   sigma    device float32 [problems][r] (out, the top singular values), or NULL
+ *   iters    subspace iterations; 0 selects the default (24)
+ *   workspace  device, 16-byte aligned, >= lla_fit_codec_workspace_bytes() bytes;
+ *            its first word is a status word (lla_workspace_flags): bit 3 (8)
+ *            means a Cholesky pivot was not positive (a rank-deficient block;
+ *            the result is then not reliable).
+ * Requires 1 <= r <= min(n, S) (else LLA_ERR_INVALID_ARG) and a block of at
+ * most 1024 columns with min(n, S) <= 32768 (else LLA_ERR_UNSUPPORTED_SHAPE).
+ * lla_fit_codec_workspace_bytes returns 0 for arguments lla_fit_codec rejects.
+ */
+size_t lla_fit_codec_workspace_bytes(int problems, int n, int S, int r);
+lla_status lla_fit_codec(int problems, int n, int S, int r, const float* X, float* mu, float* w_down,
+                         float* sigma, int iters, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
  * lla_workspace_flags — read the device status word of a decode workspace
  * (synchronises `stream`).  Bit 0: a seq_len was above max_tokens (clamped);
  * bit 1: a key or query position was outside [0, max_pos) (clamped).  The

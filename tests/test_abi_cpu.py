@@ -79,3 +79,16 @@ def test_codec_shape_mismatch_is_caught_before_the_abi():
     z = lambda *s: __import__("numpy").zeros(s)  # noqa: E731
     with pytest.raises(ValueError):
         lla.Codec(d, z(1, 1, 8, 3), z(1, 1, 8, 2), z(1, 1, 2, 4, 2), z(1, 1, 2, 4, 2), z(1, 1, 8), z(1, 1, 8))
+
+
+def test_fit_workspace_size_rules():
+    """lla_fit_codec_workspace_bytes: zero for what lla_fit_codec rejects, else enough for the
+    fp64 Gram (m x m, m = min(n, S)) and the subspace blocks of every problem."""
+    assert lla.fit_codec_workspace_bytes(1, 10, 8, 9) == 0        # r > min(n, S)
+    assert lla.fit_codec_workspace_bytes(1, 4096, 4096, 600) == 0  # block of 1200 > 1024 columns
+    assert lla.fit_codec_workspace_bytes(0, 512, 512, 16) == 0
+    one = lla.fit_codec_workspace_bytes(1, 1024, 512, 96)
+    assert one >= 512 * 512 * 8 + 2 * 512 * 192 * 8
+    assert lla.fit_codec_workspace_bytes(3, 1024, 512, 96) > 2 * one
+    # n < S uses the n x n Gram
+    assert lla.fit_codec_workspace_bytes(1, 200, 4096, 40) < lla.fit_codec_workspace_bytes(1, 4096, 4096, 40)
