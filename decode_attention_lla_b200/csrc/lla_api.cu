@@ -389,8 +389,8 @@ lla_status lla_full_decode_attn(int H, int d_head, float rope_base, const uint16
 }
 
 size_t lla_fit_codec_workspace_bytes(int problems, int n, int S, int r) {
-    if (problems < 1 || n < 1 || S < 1 || r < 1 || r > (n < S ? n : S) || (n < S ? n : S) > 32768 ||
-        !lla_fit_shape_ok(n, S, r))
+    if (problems < 1 || problems > 65535 || n < 1 || S < 1 || r < 1 || r > (n < S ? n : S) ||
+        (n < S ? n : S) > 32768 || !lla_fit_shape_ok(n, S, r))
         return 0;
     return lla_fit_workspace_bytes_impl(problems, n, S, r);
 }
@@ -400,7 +400,7 @@ lla_status lla_fit_codec(int problems, int n, int S, int r, const float* X, floa
     if (problems < 0 || n < 1 || S < 1 || r < 1 || iters < 0) return LLA_ERR_INVALID_ARG;
     const int m = n < S ? n : S;
     if (r > m) return LLA_ERR_INVALID_ARG;
-    if (m > 32768 || !lla_fit_shape_ok(n, S, r)) return LLA_ERR_UNSUPPORTED_SHAPE;
+    if (m > 32768 || problems > 65535 || !lla_fit_shape_ok(n, S, r)) return LLA_ERR_UNSUPPORTED_SHAPE;
     if (problems == 0) return LLA_OK;
     if (!X || !mu || !w_down) return LLA_ERR_INVALID_ARG;
     if (!workspace) return LLA_ERR_WORKSPACE;

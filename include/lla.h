@@ -321,7 +321,8 @@ lla_status lla_decode_attn_self(const lla_codec* codec, const uint16_t* store, i
  *            means a Cholesky pivot was not positive (a rank-deficient block;
  *            the result is then not reliable).
  * Requires 1 <= r <= min(n, S) (else LLA_ERR_INVALID_ARG) and a block of at
- * most 1024 columns with min(n, S) <= 32768 (else LLA_ERR_UNSUPPORTED_SHAPE).
+ * most 1024 columns with min(n, S) <= 32768 and problems <= 65535 (else
+ * LLA_ERR_UNSUPPORTED_SHAPE).
  * lla_fit_codec_workspace_bytes returns 0 for arguments lla_fit_codec rejects.
  */
 size_t lla_fit_codec_workspace_bytes(int problems, int n, int S, int r);

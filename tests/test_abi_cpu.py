@@ -87,6 +87,7 @@ def test_fit_workspace_size_rules():
     assert lla.fit_codec_workspace_bytes(1, 10, 8, 9) == 0        # r > min(n, S)
     assert lla.fit_codec_workspace_bytes(1, 4096, 4096, 600) == 0  # block of 1200 > 1024 columns
     assert lla.fit_codec_workspace_bytes(0, 512, 512, 16) == 0
+    assert lla.fit_codec_workspace_bytes(65536, 64, 64, 4) == 0  # problems index a grid dimension
     one = lla.fit_codec_workspace_bytes(1, 1024, 512, 96)
     assert one >= 512 * 512 * 8 + 2 * 512 * 192 * 8
     assert lla.fit_codec_workspace_bytes(3, 1024, 512, 96) > 2 * one
