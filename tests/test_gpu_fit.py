@@ -124,3 +124,27 @@ def test_fit_argument_errors():
         lla.fit_codec(4, 512, 512, 32, buf, buf, buf, None, ws)
     assert e.value.status == 6
     lla.fit_codec(0, 512, 512, 32, buf, buf, buf, None, ws)  # no problems: nothing to do
+
+
+def test_fit_full_size_sampled():
+    """All 384 (layer, head) problems of the ratio-4 V axis (1024 stacks of S = 512, r = 160) in one
+    call, as bench.py --mode fit runs them: four distinct seeded sets repeated over the batch.  Each
+    problem starts its iteration from its own pseudo-random block, so repeats agree to the
+    iteration's accuracy; one of each set is checked against the oracle."""
+    P, n, T, d, R, r = 384, 1024, 4, 128, 24, 160
+    base = _stacks("fit/fullsize", 4, n, T, d, R, 1e-2)
+    X = np.concatenate([base] * (P // 4))
+    mu_g, W_g, sig_g, flags = _fit_gpu(X, r)
+    assert flags == 0
+    for p in (0, 1, 2, 3):
+        Xp = base[p].astype(np.float64)
+        mu_o, W_o, s_o = O.fit_codec_svd(Xp, r)
+        for rep in (p + 4, p + 4 * 57, p + 4 * 95):
+            assert np.array_equal(mu_g[rep], mu_g[p])
+            assert np.abs(sig_g[rep] - sig_g[p]).max() <= 4e-6 * s_o[0]
+        assert np.abs(mu_g[p] - mu_o).max() <= 1e-6 * np.abs(mu_o).max() + 1e-7
+        assert np.abs(sig_g[p] - s_o[:r]).max() <= 2e-6 * s_o[0]
+        Xc = Xp - mu_o
+        e_gpu = np.linalg.norm(Xc - Xc @ W_g[p] @ W_g[p].T) ** 2
+        e_opt = float(np.sum(s_o[r:] ** 2))
+        assert e_gpu - e_opt <= 1e-5 * e_opt + 1e-6 * float(np.sum(s_o ** 2))

@@ -82,3 +82,33 @@ def test_full_decode_argument_errors():
     with pytest.raises(lla.LLAError) as e:  # sequence stride shorter than one sequence
         lla.full_decode_attn(16, 128, 10000.0, p, p, 100, 2, 4, p, p, p, 0.1, p, ws)
     assert e.value.status == 1
+
+
+def test_full_decode_full_size_sampled():
+    """The comparator at the bench's size and launch configuration: batch 32 x 4096 x 16 heads, one
+    (layer, loop) slice of a cache with a larger sequence stride, one persistent CTA per SM;
+    sampled sequences (one ragged) checked against the oracle."""
+    B, H, d, N = 32, 16, 128, 4096
+    cap = N + 1
+    stride = 2 * cap * H * d  # two slices per sequence: the call reads the second
+    g = torch.Generator(device=DEV)
+    g.manual_seed(syn.sub_seed("full/fullsize"))
+    K = torch.empty(B * stride, dtype=torch.bfloat16, device=DEV).normal_(generator=g)
+    V = torch.empty(B * stride, dtype=torch.bfloat16, device=DEV).normal_(generator=g)
+    q = torch.empty(B, H, d, device=DEV).normal_(generator=g)
+    lens = torch.full((B,), N, dtype=torch.int32, device=DEV)
+    lens[17] = N - 333
+    qpos = lens + 1
+    out = torch.full((B, H, d), float("nan"), device=DEV)
+    ws = torch.empty(lla.full_decode_workspace_bytes(H, d, B), dtype=torch.uint8, device=DEV)
+    off = cap * H * d
+    scale = 1 / math.sqrt(d)
+    lla.full_decode_attn(H, d, 10000.0, K.data_ptr() + 2 * off, V.data_ptr() + 2 * off, stride, B, cap, q, qpos, lens,
+                         scale, out, ws)
+    torch.cuda.synchronize()
+    assert lla.workspace_flags(ws) == 0
+    sample = [0, 17, 31]
+    kv = lambda T: T.view(B, 2, H, cap, d)[sample, 1].float().cpu().numpy().astype(np.float64).transpose(0, 2, 1, 3)
+    ref = O.full_decode(q[sample].cpu().numpy().astype(np.float64), kv(K), kv(V), lens[sample].cpu().numpy(),
+                        qpos[sample].cpu().numpy(), scale, 10000.0)
+    assert_close(out[sample].cpu().numpy().astype(np.float64), ref, "full size sampled")
