@@ -26,7 +26,7 @@
 //
 // The iteration is the approximation: singular values and the fitted subspace converge as
 // (lambda_{k+1} / lambda_r)^iters; 24 iterations (the default) reach ~1e-8 relative on the seeded smooth
-// stacks (rank-R trajectories plus noise) this build tests with.  Every kernel is plain CUDA-core
+// stacks (rank-R trajectories plus noise) of the test configurations.  Every kernel is plain CUDA-core
 // fp64 (the work is a few GFLOP per problem, dominated by latency of the small factorizations).
 #include <math.h>
 #include <stdint.h>

@@ -14,7 +14,7 @@ is the "Technical Summary" page about the same paper.
 Everything is plain NumPy in float64.  A library matmul or SVD serves as a
 step; nothing is blocked, fused or reordered beyond what the equations state.
 
-Readings of points the paper leaves open (each also listed in the design doc):
+Readings of points the paper leaves open:
 
 * RoPE convention: rotate-half pairs (i, i + d/2), frequencies
   theta_i = base ** (-2 i / d).  The paper only cites Su et al. for RoPE.
