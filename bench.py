@@ -343,15 +343,16 @@ def run_ours(a, cfg):
     impl = {"auto": lla.IMPL_AUTO, "simt": lla.IMPL_SIMT, "tc": lla.IMPL_TC}[a.kernel]
     scale = 1.0 / math.sqrt(d)
     kernel_name = a.kernel
-    def decode_call(layer, t, q, ks, vs, impl, ev):
+    def decode_call(layer, t, q, ks, vs, impl, ev, o=None):
+        o = out if o is None else o
         if table is not None:
-            lla.decode_attn_paged(codec, store, B * pages, table, pages, B, layer, t, q, qpos, lens, scale, out, ws,
+            lla.decode_attn_paged(codec, store, B * pages, table, pages, B, layer, t, q, qpos, lens, scale, o, ws,
                                   k_self=ks, v_self=vs, impl=impl, events=ev)
         elif ks is not None:
-            lla.decode_attn_self(codec, store, B, cap, layer, t, q, qpos, lens, ks, vs, scale, out, ws, impl=impl,
+            lla.decode_attn_self(codec, store, B, cap, layer, t, q, qpos, lens, ks, vs, scale, o, ws, impl=impl,
                                  events=ev)
         else:
-            lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, out, ws, impl=impl, events=ev)
+            lla.decode_attn(codec, store, B, cap, layer, t, q, qpos, lens, scale, o, ws, impl=impl, events=ev)
 
     if a.kernel == "auto":  # find which kernel "auto" runs
         try:
@@ -361,32 +362,62 @@ def run_ours(a, cfg):
             kernel_name = "simt"
         impl = {"tc": lla.IMPL_TC, "simt": lla.IMPL_SIMT}[kernel_name]
 
-    def step(events=None, host=None):
+    def step(events=None):
         k = 0
         for t in range(T):
             for layer in range(D):
-                q = q_all[t, layer]
-                if host is not None:
-                    q = host["q_dev"]
-                    q.copy_(host["q"][t, layer], non_blocking=True)
                 ev = events[k] if events is not None else None
                 ks = vs = None
                 if kv_self is not None:
-                    kv = kv_self[t, layer]
-                    if host is not None:
-                        kv = host["kv_dev"]
-                        kv.copy_(host["kv"][t, layer], non_blocking=True)
-                    ks, vs = kv[0], kv[1]
-                decode_call(layer, t, q, ks, vs, impl, ev)
-                if host is not None:
-                    host["out"][t, layer].copy_(out, non_blocking=True)
+                    ks, vs = kv_self[t, layer][0], kv_self[t, layer][1]
+                decode_call(layer, t, q_all[t, layer], ks, vs, impl, ev)
                 k += 1
-        if host is not None:
-            x_new.copy_(host["x"], non_blocking=True)
+        encode_step(x_new)
+
+    def encode_step(x):
         if table is not None:
-            lla.encode_paged(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B * pages, table, pages, B)
+            lla.encode_paged(codec, x, B, 0, D, seq_idx, tok_idx, store, B * pages, table, pages, B)
         else:
-            lla.encode(codec, x_new, B, 0, D, seq_idx, tok_idx, store, B, cap)
+            lla.encode(codec, x, B, 0, D, seq_idx, tok_idx, store, B, cap)
+
+    def step_e2e(host):
+        """One step through host buffers: every call's query (and self-slot K/V) goes up from pinned
+        memory and its output comes back, and the step's new-token stacks go up.  The copies run on
+        a copy-in and a copy-out stream beside the compute stream, into double-buffered device
+        slots ordered by events, so the transfers of neighbouring calls overlap the decode."""
+        cs = torch.cuda.current_stream(dev)
+        cin, cout = host["cin"], host["cout"]
+        with torch.cuda.stream(cin):  # this step's new-token stacks, once the last encode read them
+            cin.wait_event(host["x_free"])
+            x_new.copy_(host["x"], non_blocking=True)
+            host["x_ready"].record(cin)
+        k = 0
+        for t in range(T):
+            for layer in range(D):
+                sl = k % 2
+                with torch.cuda.stream(cin):
+                    cin.wait_event(host["done"][sl])  # the decode two calls back has read this slot
+                    host["q_dev"][sl].copy_(host["q"][t, layer], non_blocking=True)
+                    if kv_self is not None:
+                        host["kv_dev"][sl].copy_(host["kv"][t, layer], non_blocking=True)
+                    host["ready"][sl].record(cin)
+                cs.wait_event(host["ready"][sl])
+                cs.wait_event(host["out_free"][sl])  # its output two calls back has been copied out
+                ks = vs = None
+                if kv_self is not None:
+                    ks, vs = host["kv_dev"][sl][0], host["kv_dev"][sl][1]
+                decode_call(layer, t, host["q_dev"][sl], ks, vs, impl, None, host["out_dev"][sl])
+                host["done"][sl].record(cs)
+                with torch.cuda.stream(cout):
+                    cout.wait_event(host["done"][sl])
+                    host["out"][t, layer].copy_(host["out_dev"][sl], non_blocking=True)
+                    host["out_free"][sl].record(cout)
+                k += 1
+        cs.wait_event(host["x_ready"])
+        encode_step(x_new)
+        host["x_free"].record(cs)
+        for sl in range(2):  # the step ends when its last outputs are in host memory
+            cs.wait_event(host["out_free"][sl])
 
     for _ in range(a.warmup):
         step()
@@ -426,21 +457,26 @@ def run_ours(a, cfg):
         host = {"q": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
                 "out": torch.empty(T, D, B, H, d, dtype=torch.float32, pin_memory=True),
                 "x": torch.empty(x_shape, dtype=torch.bfloat16, pin_memory=True),
-                "q_dev": torch.empty(B, H, d, dtype=torch.float32, device=dev)}
+                "q_dev": [torch.empty(B, H, d, dtype=torch.float32, device=dev) for _ in range(2)],
+                "out_dev": [torch.empty(B, H, d, dtype=torch.float32, device=dev) for _ in range(2)],
+                "cin": torch.cuda.Stream(dev), "cout": torch.cuda.Stream(dev),
+                "ready": [torch.cuda.Event() for _ in range(2)], "done": [torch.cuda.Event() for _ in range(2)],
+                "out_free": [torch.cuda.Event() for _ in range(2)],
+                "x_ready": torch.cuda.Event(), "x_free": torch.cuda.Event()}
         host["q"].copy_(q_all.cpu())
         if kv_self is not None:
             host["kv"] = torch.empty(kv_self.shape, dtype=torch.float32, pin_memory=True)
             host["kv"].copy_(kv_self.cpu())
-            host["kv_dev"] = torch.empty(kv_self.shape[2:], dtype=torch.float32, device=dev)
+            host["kv_dev"] = [torch.empty(kv_self.shape[2:], dtype=torch.float32, device=dev) for _ in range(2)]
         host["x"].copy_(x_new.cpu())
-        step(host=host)
+        step_e2e(host)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(a.e2e_steps):
-            step(host=host)
+            step_e2e(host)
         e1.record()
         torch.cuda.synchronize()
         e2e_value = job_value(ctx_tokens_step, a.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), dev))
