@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         // stay adjacent in ring order and the rest of the ring keeps prefetching.
 
         float m[C::HPW], l[C::HPW], acc[C::HPW][C::VPL];
-        const float* isc_row = p.inv_scale;  // per-(b, h) score scale, re-read from L1 when needed
+        float isc[C::HPW];  // this warp's heads' score scales for the current sequence
         int len = 0;                         // clamped length of the current sequence
         uint32_t gi = 0, tile_n = 0;
         int prev_key = -1;
@@ -455,7 +455,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 }
                 prev_key = key;
                 prev_id = wk.record_id();
-                isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
+                {
+                    const float* isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
+#pragma unroll
+                    for (int hw = 0; hw < C::HPW; ++hw) isc[hw] = __ldg(isc_row + hf + C::WPQ * hw);
+                }
                 len = __ldg(p.lens + wk.b);
             }
             const int valid = min(kTile, len - wk.t * kTile);
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                         }
                     }
                     const float2 sp = f2_unpack(s01), sq = f2_unpack(s23);
-                    const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * __ldg(isc_row + hl) : -INFINITY;
+                    const float s2 = row_ok ? ((sp.x + sp.y) + (sq.x + sq.y) + bias) * isc[hw] : -INFINITY;
                     // ---- online softmax in base 2
                     const float m_new = fmaxf(m[hw], warp_max(s2));
                     const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m[hw] - m_new);
