@@ -35,6 +35,7 @@ CASES = [
     (2, 1024, 4, 128, 24, 1e-2, 96),  # the ratio-4 K rank at S = 512
     (1, 1024, 4, 128, 24, 1e-2, 160), # the ratio-4 V rank
     (2, 256, 1, 2048, 24, 1e-2, 64),  # a 2D-like stack over 16 heads x 128 (S = 2048), n < S
+    (2, 40, 2, 8, 3, 1e-3, 1),        # rank 1; the block is the whole space (k = m = 16)
 ]
 
 

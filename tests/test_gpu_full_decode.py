@@ -54,7 +54,8 @@ def _run(kb, vb, layer, B, L, N, H, d, q, qpos, lens, scale, num_ctas=0):
 
 
 @pytest.mark.parametrize("c", [dict(B=3, L=1, N=520, H=16, lens=[520, 0, 129]),
-                               dict(B=4, L=2, N=300, H=3, lens=[1, 300, 255, 77])])
+                               dict(B=4, L=2, N=300, H=3, lens=[1, 300, 255, 77]),
+                               dict(B=2, L=1, N=1, H=1, lens=[1, 0])])  # one cached token: out = v_0
 def test_full_decode_matches_oracle(c):
     B, L, N, H, d = c["B"], c["L"], c["N"], c["H"], 128
     tag = f"full/{B}/{H}"
