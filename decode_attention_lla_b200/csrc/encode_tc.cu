@@ -1,12 +1,13 @@
 // Tensor-core LLA encode: c = (x - mu) W_down = x W_down - b  [LLA §3 eq. (2)].
 //
-// One CTA per (128-token tile, layer, head): the loop stacks x of the tile
-// (K axis and V axis, S = T*d_head each, or T*H*d_head for LLA-2D) are the A
-// operand and W_down^T of the two axes the B operands of tcgen05.mma
-// (bf16 in, fp32 accumulators in TMEM: r_k columns for K, r_v for V).  K is
-// walked in 64-element chunks staged by TMA with the 128-byte swizzle into a
-// ring of shared-memory stages.  Four epilogue warps (thread = token row)
-// subtract b = mu W_down, round to bf16 (nearest-even) and write the token's
+// Persistent CTAs over the work items (128-token tile, layer, head), slot-major so that the CTAs
+// running at the same time share W_down's tiles in L2.  For an item, the loop stacks x of the
+// tile (K axis and V axis, S = T*d_head each, or T*H*d_head for LLA-2D) are the A operand and
+// W_down^T of the two axes the B operands of tcgen05.mma (bf16 in, fp32 accumulators in TMEM:
+// r_k columns for K, r_v for V).  K is walked in 64-element chunks staged by TMA with the
+// 128-byte swizzle into a ring of shared-memory stages that runs on across items.  Two TMEM
+// accumulator buffers let the MMAs of the next item run while four epilogue warps (thread =
+// token row) subtract b = mu W_down, round to bf16 (nearest-even) and write each token's
 // K || V latent row to the store slot (seq_idx[i], tok_idx[i]).
 //
 //   warp 0  TMA producer        warp 1  TMEM allocator + MMA issuer
@@ -47,13 +48,15 @@ struct ECfg {
     static constexpr int NST2 = (kSmemLimit / 2 - 2048) / STAGE;
     static constexpr int NST1 = (kSmemLimit - 2048) / STAGE;
     static constexpr int NST = NST2 >= 2 ? (NST2 > 4 ? 4 : NST2) : (NST1 > 4 ? 4 : NST1);
+    static constexpr int CTAS_PER_SM = NST2 >= 2 ? 2 : 1;
     static constexpr int SMEM = 1024 + NST * STAGE + 1024;
     static constexpr int VCOL = (RK + 31) / 32 * 32;  // TMEM column of the V accumulator
-    static constexpr int TMEM_COLS = pow2_at_least(VCOL + RV);
+    static constexpr int ACC_COLS = pow2_at_least(VCOL + RV);  // one accumulator buffer
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;              // two: epilogue and MMA overlap
     static constexpr uint32_t IDESC_K = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(RK >> 3) << 17) | (uint32_t(128 >> 4) << 24);
     static constexpr uint32_t IDESC_V = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(RV >> 3) << 17) | (uint32_t(128 >> 4) << 24);
     static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= 256 && RV <= 256, "ranks");
-    static_assert(TMEM_COLS <= 512, "TMEM");
+    static_assert(TMEM_COLS * CTAS_PER_SM <= 512, "TMEM");
     static_assert(SMEM <= kSmemLimit, "shared memory");
 };
 
@@ -64,7 +67,7 @@ struct EncParams {
     const float* bias_k;  // [D][Hg][r_k]
     const float* bias_v;
     uint32_t* status;
-    int n, layer_begin, num_layers, Hg, S, D, batch, max_tokens;
+    int n, layer_begin, num_layers, Hg, S, D, batch, max_tokens, ntiles, nitems;
     size_t row;  // elements per (sequence, layer, token) row of the store
     lla_store_map smap;
 };
@@ -84,22 +87,27 @@ __global__ void __launch_bounds__(kThreads) encode_tc_kernel(const __grid_consta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NST * C::STAGE);
     uint64_t* full = bars;                 // [NST]
     uint64_t* empty = bars + C::NST;       // [NST]
-    uint64_t* acc_full = bars + 2 * C::NST;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* acc_full = bars + 2 * C::NST;  // [2] an item's accumulators complete
+    uint64_t* acc_empty = acc_full + 2;      // [2] read out by the four epilogue warps
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x;
-    const int slot = blockIdx.y;  // L * Hg + h
-    const int L = slot / p.Hg, h = slot - L * p.Hg;
-    const int layer = p.layer_begin + L;
     const int nk = p.S / kKc;
+    // work item it -> (slot = L * Hg + h, tile): slot-major
+    auto item = [&](int it, int& tile, int& slot) {
+        slot = it / p.ntiles;
+        tile = it - slot * p.ntiles;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NST; ++i) {
             mbar_init(full + i, 1);
             mbar_init(empty + i, 1);
         }
-        mbar_init(acc_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(acc_full + i, 1);
+            mbar_init(acc_empty + i, 4);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -117,34 +125,41 @@ __global__ void __launch_bounds__(kThreads) encode_tc_kernel(const __grid_consta
             prefetch_tensormap(&wkmap);
             prefetch_tensormap(&wvmap);
             const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
-            const int wrow_k = (layer * p.Hg + h) * C::RK, wrow_v = (layer * p.Hg + h) * C::RV;
             int issued = 0;
-            for (int kc = 0; kc < nk; ++kc) {
-                const int s = kc % C::NST, round = kc / C::NST;
-                if (round > 0 && !mbar_wait(empty + s, (round - 1) & 1, p.status, 4u, 20)) break;
-                uint8_t* st = smem + size_t(s) * C::STAGE;
-                mbar_expect_tx(full + s, C::STAGE);
-                // x: dims (S, slot = (L*Hg + h)*2 + axis, token): one box per axis
-                for (int axis = 0; axis < 2; ++axis)
+            bool ok = true;
+            for (int it = blockIdx.x; it < p.nitems && ok; it += gridDim.x) {
+                int tile, slot;
+                item(it, tile, slot);
+                const int L = slot / p.Hg, h = slot - L * p.Hg;
+                const int layer = p.layer_begin + L;
+                const int wrow_k = (layer * p.Hg + h) * C::RK, wrow_v = (layer * p.Hg + h) * C::RV;
+                for (int kc = 0; kc < nk; ++kc) {
+                    const int s = issued % C::NST, round = issued / C::NST;
+                    if (round > 0 && !(ok = mbar_wait(empty + s, (round - 1) & 1, p.status, 4u, 20))) break;
+                    uint8_t* st = smem + size_t(s) * C::STAGE;
+                    mbar_expect_tx(full + s, C::STAGE);
+                    // x: dims (S, slot = (L*Hg + h)*2 + axis, token): one box per axis
+                    for (int axis = 0; axis < 2; ++axis)
+                        asm volatile(
+                            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                            " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st + axis * C::A_BYTES)),
+                            "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(kc * kKc), "r"(slot * 2 + axis),
+                            "r"(tile * kTok), "r"(smem_u32(full + s)), "l"(pol_x)
+                            : "memory");
                     asm volatile(
-                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-                        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st + axis * C::A_BYTES)),
-                        "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(kc * kKc), "r"(slot * 2 + axis), "r"(tile * kTok),
-                        "r"(smem_u32(full + s)), "l"(pol_x)
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES)),
+                        "l"(reinterpret_cast<uint64_t>(&wkmap)), "r"(kc * kKc), "r"(wrow_k), "r"(smem_u32(full + s)),
+                        "l"(pol_w)
                         : "memory");
-                asm volatile(
-                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-                    " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES)),
-                    "l"(reinterpret_cast<uint64_t>(&wkmap)), "r"(kc * kKc), "r"(wrow_k), "r"(smem_u32(full + s)),
-                    "l"(pol_w)
-                    : "memory");
-                asm volatile(
-                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-                    " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES + C::BK_BYTES)),
-                    "l"(reinterpret_cast<uint64_t>(&wvmap)), "r"(kc * kKc), "r"(wrow_v), "r"(smem_u32(full + s)),
-                    "l"(pol_w)
-                    : "memory");
-                ++issued;
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+                        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(st + 2 * C::A_BYTES + C::BK_BYTES)),
+                        "l"(reinterpret_cast<uint64_t>(&wvmap)), "r"(kc * kKc), "r"(wrow_v), "r"(smem_u32(full + s)),
+                        "l"(pol_w)
+                        : "memory");
+                    ++issued;
+                }
             }
             // drain: no copy in flight at exit
             for (int s = 0; s < C::NST && s < issued; ++s) {
@@ -155,80 +170,101 @@ __global__ void __launch_bounds__(kThreads) encode_tc_kernel(const __grid_consta
     } else if (warp == 1) {
         if (elect_one()) {
             bool ok = true;
-            for (int kc = 0; kc < nk && ok; ++kc) {
-                const int s = kc % C::NST, round = kc / C::NST;
-                if (!(ok = mbar_wait(full + s, round & 1, p.status, 4u, 22))) break;
+            int consumed = 0, j = 0;
+            for (int it = blockIdx.x; it < p.nitems && ok; it += gridDim.x, ++j) {
+                const int buf = j & 1, use = j >> 1;
+                if (use > 0 && !(ok = mbar_wait(acc_empty + buf, (use - 1) & 1, p.status, 4u, 25))) break;
                 tc_fence_after();
-                const uint32_t ak = smem_u32(smem + size_t(s) * C::STAGE), av = ak + C::A_BYTES;
-                const uint32_t bk = av + C::A_BYTES, bv = bk + C::BK_BYTES;
+                const uint32_t dk = tmem + buf * C::ACC_COLS, dv = dk + C::VCOL;
+                for (int kc = 0; kc < nk; ++kc) {
+                    const int s = consumed % C::NST, round = consumed / C::NST;
+                    if (!(ok = mbar_wait(full + s, round & 1, p.status, 4u, 22))) break;
+                    tc_fence_after();
+                    const uint32_t ak = smem_u32(smem + size_t(s) * C::STAGE), av = ak + C::A_BYTES;
+                    const uint32_t bk = av + C::A_BYTES, bv = bk + C::BK_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < kKc / 16; ++kk) {
-                    const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16_ss(tmem, sw128_kmajor_desc(ak + kk * 32), sw128_kmajor_desc(bk + kk * 32), C::IDESC_K, acc);
-                    mma_f16_ss(tmem + C::VCOL, sw128_kmajor_desc(av + kk * 32), sw128_kmajor_desc(bv + kk * 32),
-                               C::IDESC_V, acc);
+                    for (int kk = 0; kk < kKc / 16; ++kk) {
+                        const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+                        mma_f16_ss(dk, sw128_kmajor_desc(ak + kk * 32), sw128_kmajor_desc(bk + kk * 32), C::IDESC_K, acc);
+                        mma_f16_ss(dv, sw128_kmajor_desc(av + kk * 32), sw128_kmajor_desc(bv + kk * 32), C::IDESC_V, acc);
+                    }
+                    mma_commit(empty + s);
+                    ++consumed;
                 }
-                mma_commit(empty + s);
+                if (ok) mma_commit(acc_full + buf);
             }
-            mma_commit(acc_full);
-            mbar_wait(acc_full, 0, p.status, 4u, 23);
         }
     } else {
         // epilogue: warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
         const int qd = warp & 3;
         const int r = 32 * qd + lane;
-        const int i = tile * kTok + r;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.status, 4u, 24));
-        tc_fence_after();
-        const uint32_t taddr = tmem + (uint32_t(32 * qd) << 16);
-        int sq = -1, tk = -1;
-        if (i < p.n) {
-            sq = p.seq_idx[i];
-            tk = p.tok_idx[i];
-        }
-        bool write = ok && i < p.n && sq >= 0 && sq < p.batch && tk >= 0 && tk < p.max_tokens;
-        const long long ri = write ? p.smap.row_index(sq, layer, tk, p.D, p.max_tokens) : 0;
-        write = write && ri >= 0;  // a page index out of range: not written
-        uint16_t* dst = p.store + size_t(ri < 0 ? 0 : ri) * p.row + size_t(h) * (C::RK + C::RV);
-        const float* bk = p.bias_k + (size_t(layer) * p.Hg + h) * C::RK;
-        const float* bv = p.bias_v + (size_t(layer) * p.Hg + h) * C::RV;
-#pragma unroll
-        for (int a0 = 0; a0 < C::RK; a0 += 16) {
-            float v[16];
-            tmem_ld<16>(taddr + a0, v);
-            tmem_wait_ld();
-            if (write) {
-                uint4 w0, w1;
-                w0.x = pack_bf16(v[0] - bk[a0 + 0], v[1] - bk[a0 + 1]);
-                w0.y = pack_bf16(v[2] - bk[a0 + 2], v[3] - bk[a0 + 3]);
-                w0.z = pack_bf16(v[4] - bk[a0 + 4], v[5] - bk[a0 + 5]);
-                w0.w = pack_bf16(v[6] - bk[a0 + 6], v[7] - bk[a0 + 7]);
-                w1.x = pack_bf16(v[8] - bk[a0 + 8], v[9] - bk[a0 + 9]);
-                w1.y = pack_bf16(v[10] - bk[a0 + 10], v[11] - bk[a0 + 11]);
-                w1.z = pack_bf16(v[12] - bk[a0 + 12], v[13] - bk[a0 + 13]);
-                w1.w = pack_bf16(v[14] - bk[a0 + 14], v[15] - bk[a0 + 15]);
-                reinterpret_cast<uint4*>(dst + a0)[0] = w0;
-                reinterpret_cast<uint4*>(dst + a0)[1] = w1;
+        bool ok = true;
+        int j = 0;
+        for (int it = blockIdx.x; it < p.nitems && ok; it += gridDim.x, ++j) {
+            int tile, slot;
+            item(it, tile, slot);
+            const int L = slot / p.Hg, h = slot - L * p.Hg;
+            const int layer = p.layer_begin + L;
+            const int i = tile * kTok + r;
+            // the row's destination, read before the accumulators are ready
+            int sq = -1, tk = -1;
+            if (i < p.n) {
+                sq = __ldg(p.seq_idx + i);
+                tk = __ldg(p.tok_idx + i);
             }
-        }
+            const int buf = j & 1, use = j >> 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(acc_full + buf, use & 1, p.status, 4u, 24));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem + buf * C::ACC_COLS + (uint32_t(32 * qd) << 16);
+            bool write = i < p.n && sq >= 0 && sq < p.batch && tk >= 0 && tk < p.max_tokens;
+            const long long ri = write ? p.smap.row_index(sq, layer, tk, p.D, p.max_tokens) : 0;
+            write = write && ri >= 0;  // a page index out of range: not written
+            uint16_t* dst = p.store + size_t(ri < 0 ? 0 : ri) * p.row + size_t(h) * (C::RK + C::RV);
+            const float* bk = p.bias_k + (size_t(layer) * p.Hg + h) * C::RK;
+            const float* bv = p.bias_v + (size_t(layer) * p.Hg + h) * C::RV;
 #pragma unroll
-        for (int a0 = 0; a0 < C::RV; a0 += 16) {
-            float v[16];
-            tmem_ld<16>(taddr + C::VCOL + a0, v);
-            tmem_wait_ld();
-            if (write) {
-                uint4 w0, w1;
-                w0.x = pack_bf16(v[0] - bv[a0 + 0], v[1] - bv[a0 + 1]);
-                w0.y = pack_bf16(v[2] - bv[a0 + 2], v[3] - bv[a0 + 3]);
-                w0.z = pack_bf16(v[4] - bv[a0 + 4], v[5] - bv[a0 + 5]);
-                w0.w = pack_bf16(v[6] - bv[a0 + 6], v[7] - bv[a0 + 7]);
-                w1.x = pack_bf16(v[8] - bv[a0 + 8], v[9] - bv[a0 + 9]);
-                w1.y = pack_bf16(v[10] - bv[a0 + 10], v[11] - bv[a0 + 11]);
-                w1.z = pack_bf16(v[12] - bv[a0 + 12], v[13] - bv[a0 + 13]);
-                w1.w = pack_bf16(v[14] - bv[a0 + 14], v[15] - bv[a0 + 15]);
-                reinterpret_cast<uint4*>(dst + C::RK + a0)[0] = w0;
-                reinterpret_cast<uint4*>(dst + C::RK + a0)[1] = w1;
+            for (int a0 = 0; a0 < C::RK; a0 += 16) {
+                float v[16];
+                tmem_ld<16>(taddr + a0, v);
+                tmem_wait_ld();
+                if (write) {
+                    uint4 w0, w1;
+                    w0.x = pack_bf16(v[0] - bk[a0 + 0], v[1] - bk[a0 + 1]);
+                    w0.y = pack_bf16(v[2] - bk[a0 + 2], v[3] - bk[a0 + 3]);
+                    w0.z = pack_bf16(v[4] - bk[a0 + 4], v[5] - bk[a0 + 5]);
+                    w0.w = pack_bf16(v[6] - bk[a0 + 6], v[7] - bk[a0 + 7]);
+                    w1.x = pack_bf16(v[8] - bk[a0 + 8], v[9] - bk[a0 + 9]);
+                    w1.y = pack_bf16(v[10] - bk[a0 + 10], v[11] - bk[a0 + 11]);
+                    w1.z = pack_bf16(v[12] - bk[a0 + 12], v[13] - bk[a0 + 13]);
+                    w1.w = pack_bf16(v[14] - bk[a0 + 14], v[15] - bk[a0 + 15]);
+                    reinterpret_cast<uint4*>(dst + a0)[0] = w0;
+                    reinterpret_cast<uint4*>(dst + a0)[1] = w1;
+                }
             }
+#pragma unroll
+            for (int a0 = 0; a0 < C::RV; a0 += 16) {
+                float v[16];
+                tmem_ld<16>(taddr + C::VCOL + a0, v);
+                tmem_wait_ld();
+                if (write) {
+                    uint4 w0, w1;
+                    w0.x = pack_bf16(v[0] - bv[a0 + 0], v[1] - bv[a0 + 1]);
+                    w0.y = pack_bf16(v[2] - bv[a0 + 2], v[3] - bv[a0 + 3]);
+                    w0.z = pack_bf16(v[4] - bv[a0 + 4], v[5] - bv[a0 + 5]);
+                    w0.w = pack_bf16(v[6] - bv[a0 + 6], v[7] - bv[a0 + 7]);
+                    w1.x = pack_bf16(v[8] - bv[a0 + 8], v[9] - bv[a0 + 9]);
+                    w1.y = pack_bf16(v[10] - bv[a0 + 10], v[11] - bv[a0 + 11]);
+                    w1.z = pack_bf16(v[12] - bv[a0 + 12], v[13] - bv[a0 + 13]);
+                    w1.w = pack_bf16(v[14] - bv[a0 + 14], v[15] - bv[a0 + 15]);
+                    reinterpret_cast<uint4*>(dst + C::RK + a0)[0] = w0;
+                    reinterpret_cast<uint4*>(dst + C::RK + a0)[1] = w1;
+                }
+            }
+            // this warp's lanes of the buffer are read: the MMAs of the item after next may use it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + buf);
         }
     }
     tc_fence_before();
@@ -315,8 +351,13 @@ lla_status run_encode(const lla_codec* c, const uint16_t* x, int n, int layer_be
     p.max_tokens = max_tokens;
     p.row = size_t(ds.r_k + ds.r_v) * Hg;
     p.smap = smap;
+    p.ntiles = (n + kTok - 1) / kTok;
+    const long long items = (long long)p.ntiles * num_layers * Hg;
+    if (items > 0x7fffffffLL) return LLA_ERR_UNSUPPORTED_SHAPE;
+    p.nitems = int(items);
     LLA_CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-    dim3 grid((n + kTok - 1) / kTok, num_layers * Hg);
+    const long long slots = (long long)lla_num_sms() * C::CTAS_PER_SM;
+    const int grid = int(items < slots ? items : slots);
     encode_tc_kernel<C><<<grid, kThreads, C::SMEM, stream>>>(xmap, wkmap, wvmap, p);
     LLA_CUDA_TRY(cudaGetLastError());
     return LLA_OK;
