@@ -414,23 +414,38 @@ __global__ void __launch_bounds__(1024) fit_jacobi_kernel(double* Hm, double* Vm
                 }
             }
             __syncthreads();
-            // columns p, q of every row: H <- H J, V <- V J, one row at a time per warp through
-            // its shared-memory row buffer (contiguous loads and stores)
+            // columns p, q of every row: H <- H J, V <- V J, two rows at a time per warp through
+            // its shared-memory row buffers (contiguous loads and stores, both rows in flight)
             if (warp < col_warps) {
-                double* rb = rowbuf + size_t(warp) * kk;
-                for (int i = warp; i < 2 * kk; i += col_warps) {
-                    double* row = i < kk ? H + size_t(i) * kk : V + size_t(i - kk) * kk;
-                    for (int j = lane; j < kk; j += 32) rb[j] = row[j];
+                double* rb0 = rowbuf + size_t(2 * warp) * kk;
+                double* rb1 = rb0 + kk;
+                for (int i = warp; i < 2 * kk; i += 2 * col_warps) {
+                    const int i1 = i + col_warps;
+                    const bool two = i1 < 2 * kk;
+                    double* row0 = i < kk ? H + size_t(i) * kk : V + size_t(i - kk) * kk;
+                    double* row1 = !two ? row0 : (i1 < kk ? H + size_t(i1) * kk : V + size_t(i1 - kk) * kk);
+                    for (int j = lane; j < kk; j += 32) {
+                        rb0[j] = row0[j];
+                        if (two) rb1[j] = row1[j];
+                    }
                     __syncwarp();
                     for (int a = lane; a < na; a += 32) {
                         const int p = act_p[a], q = act_q[a];
                         const double c = act_c[a], sn = act_s[a];
-                        const double x = rb[p], y = rb[q];
-                        rb[p] = c * x - sn * y;
-                        rb[q] = sn * x + c * y;
+                        const double x0 = rb0[p], y0 = rb0[q];
+                        rb0[p] = c * x0 - sn * y0;
+                        rb0[q] = sn * x0 + c * y0;
+                        if (two) {
+                            const double x1 = rb1[p], y1 = rb1[q];
+                            rb1[p] = c * x1 - sn * y1;
+                            rb1[q] = sn * x1 + c * y1;
+                        }
                     }
                     __syncwarp();
-                    for (int j = lane; j < kk; j += 32) row[j] = rb[j];
+                    for (int j = lane; j < kk; j += 32) {
+                        row0[j] = rb0[j];
+                        if (two) row1[j] = rb1[j];
+                    }
                     __syncwarp();
                 }
             }
@@ -587,8 +602,8 @@ lla_status lla_fit(int P, int n, int S, int r, const float* X, float* mu_out, fl
     // row per warp (at most ~200 KB)
     const int tri_warps = (200 * 1024) / (8 * k) < 32 ? (200 * 1024) / (8 * k) : 32;
     const size_t tri_smem = size_t(tri_warps) * k * sizeof(double);
-    const int col_warps = (200 * 1024) / (8 * kk) < 32 ? (200 * 1024) / (8 * kk) : 32;
-    const size_t jac_smem = size_t(col_warps) * kk * sizeof(double);
+    const int col_warps = (200 * 1024) / (16 * kk) < 32 ? (200 * 1024) / (16 * kk) : 32;
+    const size_t jac_smem = size_t(2 * col_warps) * kk * sizeof(double);
     LLA_CUDA_TRY(cudaFuncSetAttribute(fit_trinv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tri_smem)));
     LLA_CUDA_TRY(cudaFuncSetAttribute(fit_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(jac_smem)));
 
