@@ -388,6 +388,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 
         float m[C::HPW], l[C::HPW], acc[C::HPW][C::VPL];
         float isc[C::HPW];  // this warp's heads' score scales for the current sequence
+        // the next sequence's length and scales, loaded at the previous sequence change so that
+        // their latency is off the first tile (narrow rows only: the wide-row warps carry 16
+        // heads and have no registers to spare)
+        constexpr bool kPrefetchSeq = !C::WIDE;
+        int pf_b = -1, pf_len = 0;
+        float pf_isc[kPrefetchSeq ? C::HPW : 1];
         int len = 0;                         // clamped length of the current sequence
         uint32_t gi = 0, tile_n = 0;
         int prev_key = -1;
@@ -455,12 +461,25 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
                 }
                 prev_key = key;
                 prev_id = wk.record_id();
-                {
+                if (kPrefetchSeq && pf_b == wk.b) {
+#pragma unroll
+                    for (int hw = 0; hw < C::HPW; ++hw) isc[hw] = pf_isc[kPrefetchSeq ? hw : 0];
+                    len = pf_len;
+                } else {
                     const float* isc_row = p.inv_scale + size_t(wk.b) * C::H + wk.p * C::HC;
 #pragma unroll
                     for (int hw = 0; hw < C::HPW; ++hw) isc[hw] = __ldg(isc_row + hf + C::WPQ * hw);
+                    len = __ldg(p.lens + wk.b);
                 }
-                len = __ldg(p.lens + wk.b);
+                if (kPrefetchSeq) {
+                    pf_b = wk.b + 1 < p.B ? wk.b + 1 : -1;
+                    if (pf_b >= 0) {
+                        const float* isc_row = p.inv_scale + size_t(pf_b) * C::H + wk.p * C::HC;
+#pragma unroll
+                        for (int hw = 0; hw < C::HPW; ++hw) pf_isc[kPrefetchSeq ? hw : 0] = __ldg(isc_row + hf + C::WPQ * hw);
+                        pf_len = __ldg(p.lens + pf_b);
+                    }
+                }
             }
             const int valid = min(kTile, len - wk.t * kTile);
             const bool row_ok = row < valid;
