@@ -15,9 +15,9 @@
 // since the cached tokens then carry 1 - w_self of the probability.
 //
 // One CTA per (head, 8 sequences, slice of output dimensions), one warp per sequence: the rows
-// of W^V_up,t of its slice are staged in shared memory, read from global memory in their own
-// order (coalesced) and kept row-major with an odd row pitch, so that the lanes of a warp (one
-// output dimension each at a time) read distinct banks.  Small batches split d into 32-row
+// of W^V_up,t of its slice are copied asynchronously into shared memory, read from global
+// memory in their own order (coalesced) and kept row-major with an odd row pitch, so that the
+// lanes of a warp (one output dimension each at a time) read distinct banks.  Small batches split d into 32-row
 // slices to fill the machine, and every CTA of a (head, sequence) then merges the records
 // itself (cheap next to the projection); large batches keep all d rows in one CTA.
 #include <math.h>
@@ -28,8 +28,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kSeqPerCta = kThreads / 32;  // one warp per sequence
-constexpr int kMaxRowsPerLane = 8;         // output dimensions per lane and pass
-constexpr int kAC = 8;                     // latent dims per lane held in registers while merging
+constexpr int kMaxRowsPerLane = 8;         // output dimensions per lane: d <= 256
 
 // Row pitch of the staged W^V_up,t: odd, so rows i and i + 1 start in different banks.
 __host__ __device__ inline int w_pitch(int rv) { return rv | 1; }
@@ -66,8 +65,15 @@ struct RecordSet {
     int s0, hstride, hrec;
     // tensor-core kernel
     bool tc;
-    long long g0;
+    long long g0, total, groups;
     int b, part, parts, hc;
+    // did group g0 + i write its records?  Only a group with an empty tile range writes none,
+    // and there is none unless the batch has fewer tiles than there are groups.
+    __device__ bool written_group(int i) const {
+        if (!tc || total >= groups) return true;
+        const int t = int(total), gs = int(groups), g = int(g0) + i;  // total < groups: small
+        return t * (g + 1) / gs > t * g / gs;
+    }
     __device__ const float* rec(int s) const {
         if (!tc) return base + (size_t(s0 + s) * hstride + hrec) * rec_len;
         const long long id = (g0 + s / 4 + b) * parts + part;
@@ -82,6 +88,9 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
     r.tc = p.tc_P != nullptr;
     r.b = b;
     r.n = 0;
+    r.g0 = 0;
+    r.total = 0;
+    r.groups = 1;
     if (r.tc) {
         r.parts = p.tc_parts;
         r.hc = p.tc_hc;
@@ -91,6 +100,8 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
         const int tiles = p.tc_P[b + 1] - p.tc_P[b];
         const long long groups = p.tc_G / p.tc_parts;
         if (tiles == 0 || total == 0 || groups == 0) return r;
+        r.total = total;
+        r.groups = groups;
         const long long x0 = p.tc_P[b], x1 = x0 + tiles - 1;
         r.g0 = ((x0 + 1) * groups - 1) / total;
         const long long g1 = ((x1 + 1) * groups - 1) / total;
@@ -109,11 +120,20 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
     return r;
 }
 
-// One warp per (sequence, head); the CTA's eight warps share 32 rows of W^V_up,t of one head.
-__global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
+// One warp per (sequence, head); the CTA's eight warps share the rows of W^V_up,t of one head.
+// A lane holds NC latent dimensions (a = lane + 32 c, c < NC, 32 NC >= r_v) and RPL output
+// rows (32 RPL >= the CTA's rows).  The warp's loads
+// go out in as few dependent rounds as the data allows: W (asynchronous copies into shared
+// memory) and mu before the wait for the decode kernel, then the record set's bounds, then every
+// record's (m, l) together with the acc of the first kRC records; the merge and the projection
+// then run from registers and shared memory.
+template <int NC, int RPL>
+__global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
+    constexpr int kRC = NC <= 2 ? 8 : 16 / NC >= 2 ? 16 / NC : 2;  // records whose acc a lane holds at once
     const int h = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y * kSeqPerCta + warp;
+    const bool active = b < p.B;
     const int d = p.d, rv = p.r_v, pitch = w_pitch(rv);
     const int rows = d / gridDim.z;  // output dimensions of this CTA's slice (gridDim.z divides d)
     const int i0 = blockIdx.z * rows;
@@ -129,120 +149,174 @@ __global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
         w_off = ((size_t(p.layer) * p.T + p.loop) * p.H + h) * size_t(d) * rv;
         mu_off = size_t(p.layer) * p.T * p.H * d + (size_t(p.loop) * p.H + h) * d;
     }
-    const float* wg = p.w_up_v + w_off + size_t(i0) * rv;
-    const int nw = rows * rv;
-    if ((rv & 3) == 0 && (reinterpret_cast<uintptr_t>(wg) & 15) == 0) {
-        // four consecutive elements of one row per load (rv % 4 == 0: no load spans two rows)
-#pragma unroll 4
-        for (int e = 4 * threadIdx.x; e < nw; e += 4 * kThreads) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(wg + e));
-            const int r = e / rv, a = e - r * rv;
-            float* w = Ws + size_t(r) * pitch + a;
-            w[0] = v.x;
-            w[1] = v.y;
-            w[2] = v.z;
-            w[3] = v.w;
-        }
-    } else {
-#pragma unroll 4
+    {
+        // W is read in its own (coalesced) order; each element lands at its padded place
+        const float* wg = p.w_up_v + w_off + size_t(i0) * rv;
+        const int nw = rows * rv;
+        int r = threadIdx.x / rv, a = threadIdx.x - (threadIdx.x / rv) * rv;
+        const int dr = kThreads / rv, da = kThreads - (kThreads / rv) * rv;
         for (int e = threadIdx.x; e < nw; e += kThreads) {
-            const int r = e / rv, a = e - r * rv;
-            Ws[size_t(r) * pitch + a] = __ldg(wg + e);
+            lla_cp_async4(Ws + size_t(r) * pitch + a, wg + e);
+            r += dr;
+            a += da;
+            if (a >= rv) {
+                a -= rv;
+                ++r;
+            }
         }
     }
-    __syncthreads();
-    lla_grid_dependency_wait();  // W above is a constant; the records come from the decode kernel
-    if (b >= p.B) return;
+    // mu of this lane's output rows r = lane + 32 k
+    float muv[RPL];
+#pragma unroll
+    for (int k = 0; k < RPL; ++k) {
+        const int r = lane + 32 * k;
+        muv[k] = (active && r < rows) ? __ldg(p.mu_v + mu_off + i0 + r) : 0.f;
+    }
+    lla_grid_dependency_wait();  // W and mu are constants; the records come from the decode kernel
 
-    const RecordSet rs = record_set(p, b, h);
-    auto rec = [&](int s) { return rs.rec(s); };
-    const int s0 = 0, s1 = rs.n;
     const size_t bh = size_t(b) * p.H + h;
-    // self-slot logit (natural-log units, like the records' m)
-    float s_self = -INFINITY;
-    if (p.k_self) {
-        float dot = 0.f;
-        for (int i = lane; i < d; i += 32) dot = fmaf(p.q[bh * d + i], p.k_self[bh * d + i], dot);
+    float L = 0.f, w_self = 0.f;
+    if (active) {
+        const RecordSet rs = record_set(p, b, h);
+        const int n = rs.n;
+        // groups of the record set that wrote records (a group whose tile range is empty did
+        // not): one bit per group for the first 32 groups, computed directly beyond
+        uint32_t wmask = 0xffffffffu;
+        if (rs.tc) wmask = __ballot_sync(0xffffffffu, lane * 4 < n && rs.written_group(lane));
+        auto written = [&](int s) { return s / 4 < 32 ? ((wmask >> (s / 4)) & 1u) != 0 : rs.written_group(s / 4); };
+        // records go in blocks of 32, record sb + j of a block on lane j: its address, (m, l) and
+        // weight are that lane's, and reach the warp by shuffle
+        auto shfl_ptr = [&](const float* q, int j) -> const float* {
+            const uint64_t u = reinterpret_cast<uint64_t>(q);
+            const uint32_t lo = __shfl_sync(0xffffffffu, uint32_t(u), j), hi = __shfl_sync(0xffffffffu, uint32_t(u >> 32), j);
+            return reinterpret_cast<const float*>((uint64_t(hi) << 32) | lo);
+        };
+        const float* my = rs.rec(lane < n ? lane : 0);
+        // one round: (m, l) of record `lane` and the acc of records [0, kRC)
+        float m0 = -INFINITY, l0 = 0.f;
+        if (lane < n && written(lane)) {
+            m0 = my[0];
+            l0 = my[1];
+        }
+        float x0[kRC][NC];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        s_self = p.scale * dot;
-    }
-    // merged maximum and normaliser over the records (log-sum-exp); a record with l = 0
-    // saw no valid token and is skipped whatever its m holds
-    float M = s_self;
-    for (int s = s0 + lane; s < s1; s += 32) {
-        const float* r = rec(s);
-        if (r[1] > 0.f) M = fmaxf(M, r[0]);
-    }
+        for (int j = 0; j < kRC; ++j) {
+            const bool use = j < n && written(j);
+            const float* r = shfl_ptr(my, j) + 2 + lane;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    if (M != -INFINITY)
-        for (int s = s0 + lane; s < s1; s += 32) {
-            const float* r = rec(s);
-            if (r[1] > 0.f) L += r[1] * expf(r[0] - M);
+            for (int c = 0; c < NC; ++c) x0[j][c] = (use && lane + 32 * c < rv) ? r[32 * c] : 0.f;
+        }
+        // self-slot logit (natural-log units, like the records' m)
+        float s_self = -INFINITY;
+        if (p.k_self) {
+            float dot = 0.f;
+            for (int i = lane; i < d; i += 32) dot = fmaf(p.q[bh * d + i], p.k_self[bh * d + i], dot);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            s_self = p.scale * dot;
+        }
+        // log-sum-exp over the records: a lane-wise running merge, then across the warp; a
+        // record with l = 0 saw no valid token and is skipped whatever its m holds
+        float mx = -INFINITY, sx = 0.f;
+        auto merge = [&](float ms, float ls) {
+            if (!(ls > 0.f)) return;
+            if (ms > mx) {
+                sx = sx * expf(mx - ms) + ls;
+                mx = ms;
+            } else {
+                sx += ls * expf(ms - mx);
+            }
+        };
+        merge(m0, l0);
+#pragma unroll 1
+        for (int s = lane + 32; s < n; s += 32)
+            if (written(s)) {
+                const float* r = rs.rec(s);
+                merge(r[0], r[1]);
+            }
+        float M = mx;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        M = fmaxf(M, s_self);
+        L = sx > 0.f ? sx * expf(mx - M) : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float e_self = p.k_self ? expf(s_self - M) : 0.f;
+        L += e_self;
+        const float invL = L > 0.f ? 1.f / L : 0.f;
+        w_self = e_self * invL;
+        // abar = sum_s w_s acc_s with w_s = exp(m_s - M) / L
+        const float w0 = l0 > 0.f ? expf(m0 - M) * invL : 0.f;
+        float v[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) v[c] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kRC; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w0, j);
+#pragma unroll
+            for (int c = 0; c < NC; ++c) v[c] = fmaf(x0[j][c], wj, v[c]);
+        }
+#pragma unroll 1
+        for (int sb = 0; sb < n; sb += 32) {
+            const float* mine = my;
+            float wb = w0;
+            if (sb > 0) {
+                const int s = sb + lane;
+                mine = rs.rec(s < n ? s : sb);
+                wb = 0.f;
+                if (s < n && written(s) && mine[1] > 0.f) wb = expf(mine[0] - M) * invL;
+            }
+            const int nb = min(32, n - sb);
+#pragma unroll 1
+            for (int j0 = sb == 0 ? kRC : 0; j0 < nb; j0 += kRC) {
+                float x[kRC][NC];
+#pragma unroll
+                for (int j = 0; j < kRC; ++j) {
+                    const int jj = (j0 + j) & 31;
+                    const bool use = j0 + j < nb && written(sb + jj);
+                    const float* r = shfl_ptr(mine, jj) + 2 + lane;
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) x[j][c] = (use && lane + 32 * c < rv) ? r[32 * c] : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kRC; ++j) {
+                    const float wj = __shfl_sync(0xffffffffu, wb, (j0 + j) & 31);
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) v[c] = fmaf(x[j][c], wj, v[c]);
+                }
+            }
         }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float e_self = p.k_self ? expf(s_self - M) : 0.f;
-    L += e_self;
+        for (int c = 0; c < NC; ++c)
+            if (lane + 32 * c < rv) abar[lane + 32 * c] = v[c];
+    }
+    lla_cp_async_wait_all();
+    __syncthreads();  // W staged by every thread of the CTA
+    if (!active) return;
     float* o = p.out + bh * d;
     if (!(L > 0.f)) {  // empty context
         for (int r = lane; r < rows; r += 32) o[i0 + r] = 0.f;
         return;
     }
-    const float w_self = e_self / L;
-    // abar = sum_s w_s acc_s with w_s = exp(m_s - M) / L; record weights one per lane, broadcast
-    // by shuffle; lane owns latent dims a0 + lane + 32 c, kAC of them per pass over the records
-    const float invL = 1.f / L;
-    for (int a0 = 0; a0 < rv; a0 += 32 * kAC) {
-        float v[kAC];
-#pragma unroll
-        for (int c = 0; c < kAC; ++c) v[c] = 0.f;
-        for (int sb = s0; sb < s1; sb += 32) {
-            float wgt = 0.f;
-            if (sb + lane < s1) {
-                const float* r = rec(sb + lane);
-                if (r[1] > 0.f) wgt = expf(r[0] - M) * invL;
-            }
-            const int ns = min(32, s1 - sb);
-#pragma unroll 2
-            for (int j = 0; j < ns; ++j) {
-                const float wj = __shfl_sync(0xffffffffu, wgt, j);
-                if (wj == 0.f) continue;  // an empty record: its acc is not read
-                const float* r = rec(sb + j) + 2 + a0 + lane;
-#pragma unroll
-                for (int c = 0; c < kAC; ++c)
-                    if (a0 + lane + 32 * c < rv) v[c] = fmaf(r[32 * c], wj, v[c]);
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < kAC; ++c)
-            if (a0 + lane + 32 * c < rv) abar[a0 + lane + 32 * c] = v[c];
-    }
-    __syncwarp();
     // out_i = abar . W^V_up,t[i] + (1 - w_self) mu^V_t[i] + w_self v_self[i] for i = i0 + r,
-    // r = r0 + lane + 32 k; the rows of a lane keep independent accumulation chains
-    for (int r0 = 0; r0 < rows; r0 += 32 * kMaxRowsPerLane) {
-        float acc[kMaxRowsPerLane];
+    // r = lane + 32 k; the rows of a lane keep independent accumulation chains
+    float acc[RPL];
 #pragma unroll
-        for (int k = 0; k < kMaxRowsPerLane; ++k) acc[k] = 0.f;
-        const float* wr = Ws + size_t(min(r0 + lane, rows - 1)) * pitch;
-        const int nk = min(kMaxRowsPerLane, (rows - r0 + 31) / 32);
-        for (int a = 0; a < rv; ++a) {
-            const float x = abar[a];
+    for (int k = 0; k < RPL; ++k) acc[k] = 0.f;
+    const float* wr = Ws + size_t(min(lane, rows - 1)) * pitch;
+    const int nk = (rows + 31) / 32;
+    for (int a = 0; a < rv; ++a) {
+        const float x = abar[a];
 #pragma unroll
-            for (int k = 0; k < kMaxRowsPerLane; ++k)
-                if (k < nk && r0 + lane + 32 * k < rows) acc[k] = fmaf(x, wr[size_t(32 * k) * pitch + a], acc[k]);
-        }
+        for (int k = 0; k < RPL; ++k)
+            if (k < nk && lane + 32 * k < rows) acc[k] = fmaf(x, wr[size_t(32 * k) * pitch + a], acc[k]);
+    }
 #pragma unroll
-        for (int k = 0; k < kMaxRowsPerLane; ++k) {
-            const int r = r0 + lane + 32 * k;
-            if (k >= nk || r >= rows) break;
-            const int i = i0 + r;
-            const float m = __ldg(p.mu_v + mu_off + i);
-            o[i] = acc[k] + (p.k_self ? fmaf(w_self, p.v_self[bh * d + i], (1.f - w_self) * m) : m);
-        }
+    for (int k = 0; k < RPL; ++k) {
+        const int r = lane + 32 * k;
+        if (k >= nk || r >= rows) break;
+        const int i = i0 + r;
+        o[i] = acc[k] + (p.k_self ? fmaf(w_self, p.v_self[bh * d + i], (1.f - w_self) * muv[k]) : muv[k]);
     }
 }
 
@@ -275,6 +349,7 @@ lla_status lla_combine_tc(const lla_decode_call& call, const float* records, con
 
 static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) {
     const lla_codec_desc& ds = call.codec->desc;
+    if (ds.d_head > 32 * kMaxRowsPerLane || ds.r_v > 256) return LLA_ERR_UNSUPPORTED_SHAPE;
     p.w_up_v = call.codec->w_up_v;
     p.mu_v = call.codec->mu_v;
     p.out = call.out;
@@ -295,9 +370,25 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     int z = 1;
     while (ds.d_head % (64 * z) == 0 && ds.H * seq_ctas * z < 2 * lla_num_sms()) z *= 2;
     const size_t smem = (size_t(w_pitch(ds.r_v)) * (ds.d_head / z) + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
-    LLA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    void (*kernel)(CombineParams) = nullptr;
+    const bool rows4 = ds.d_head / z <= 128;
+    switch ((ds.r_v + 31) / 32) {
+#define LLA_COMBINE_CASE(nc) \
+    case nc: kernel = rows4 ? combine_kernel<nc, 4> : combine_kernel<nc, kMaxRowsPerLane>; break;
+        LLA_COMBINE_CASE(1)
+        LLA_COMBINE_CASE(2)
+        LLA_COMBINE_CASE(3)
+        LLA_COMBINE_CASE(4)
+        LLA_COMBINE_CASE(5)
+        LLA_COMBINE_CASE(6)
+        LLA_COMBINE_CASE(7)
+        LLA_COMBINE_CASE(8)
+#undef LLA_COMBINE_CASE
+        default: return LLA_ERR_UNSUPPORTED_SHAPE;
+    }
+    LLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     dim3 grid(ds.H, seq_ctas, z);
     // overlapped with the decode kernel's tail, unless an event follows that kernel for timing
-    LLA_CUDA_TRY(lla_launch(combine_kernel, grid, dim3(kThreads), smem, call.stream, call.ev_end == nullptr, p));
+    LLA_CUDA_TRY(lla_launch(kernel, grid, dim3(kThreads), smem, call.stream, call.ev_end == nullptr, p));
     return LLA_OK;
 }

@@ -651,7 +651,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 #include "decode_tc2d.cuh"
 
 // ---------------------------------------------------------------------------------------------
-// Prologue: tile plan, per-(sequence, head) M_q images, record initialisation.
+// Prologue: tile plan and per-(sequence, head) M_q images with their score scales.
 // ---------------------------------------------------------------------------------------------
 
 struct ProParams {
@@ -665,10 +665,9 @@ struct ProParams {
     int32_t* lens;
     float* inv_scale;
     uint8_t* mq;
-    float* records;
-    size_t n_record_floats;
     uint32_t* status;
     int B, D, T, H, DH, RK, RV, HG, NG, HC, GPC, max_tokens, max_pos, layer, loop, variant;
+    int pro_wps, pro_spw;  // warps per sequence, sequences per group of warps
     float scale;
     lla_store_map smap;
 };
@@ -713,132 +712,104 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         if (threadIdx.x == 0) p.P[p.B] = carry;
         return;
     }
-    // CTA (head h, SPC sequences), WPS warps per sequence (SPC * WPS = 8): this head's rows of
-    // each sequence's M_q image.  W^K_up,t of the head ([n][i], row RK = mu) is staged in shared
-    // memory once; the items of a sequence are spread over its warps so that every lane keeps
-    // its few values in registers between the max and the write.
+    // CTA (head h, run of sequences): W^K_up,t of the head ([n][i], row RK = mu) is copied once
+    // into shared memory; the warps then walk the run, pro_wps warps per sequence (its items
+    // spread over them) and pro_spw sequences per group of warps.  All the items of a lane share
+    // one 8-wide k chunk (d/8 divides 32), so per sequence the lane rotates and scales the 16
+    // entries of q it needs (its rotate-half pairs) once and keeps them in registers.
     constexpr int DH = C::DH, RK = C::RK, half = DH / 2, KC = DH / 8;
     constexpr int NITEM = (RK + 1) * KC;  // (row, 8-wide k chunk) items
-    constexpr int WPS = NITEM >= 1024 ? 8 : NITEM >= 512 ? 4 : NITEM >= 256 ? 2 : 1;
-    constexpr int SPC = 8 / WPS;
-    static_assert(DH % 4 == 0, "float4 staging");
-    extern __shared__ __align__(16) float pro_smem[];
+    static_assert(32 % KC == 0, "a lane's k chunk is the same in every item it takes");
+    static_assert(half % 8 == 0, "no k chunk straddles the rotate-half boundary");
+    extern __shared__ __align__(16) float pro_smem[];  // W^K_up,t of the head: [RK + 1][DH]
     __shared__ float red[8];
+    const int wps = p.pro_wps, sls = 8 / wps, per_cta = sls * p.pro_spw;
     const int k = blockIdx.x - 1;
-    const int sl = w / WPS, wi = w % WPS;
-    const int h = k % C::H, b = (k / C::H) * SPC + sl;
-    const bool active = b < p.B;
+    const int h = k % C::H, b_first = (k / C::H) * per_cta;
+    const int sl = w / wps, wi = w % wps;
     const size_t slot = p.variant == 0 ? (size_t(p.layer) * C::H + h) * p.T + p.loop
                                        : (size_t(p.layer) * p.T + p.loop) * C::H + h;
-    float* wt = pro_smem;
-    // W loads all issued up front (their latency overlaps the rotation of q below), stored after
-    constexpr int NW4 = (RK + 1) * DH / 4, WPT = (NW4 + 255) / 256;
-    float4 wreg[WPT];
     {
-        const float4* wg = reinterpret_cast<const float4*>(p.w_up_k_t + slot * size_t(RK + 1) * DH);
-#pragma unroll
-        for (int j = 0; j < WPT; ++j) {
-            const int e = threadIdx.x + 256 * j;
-            if (e < NW4) wreg[j] = __ldg(wg + e);
-        }
+        const float* wsrc = p.w_up_k_t + slot * size_t(RK + 1) * DH;
+        constexpr int NW4 = (RK + 1) * DH / 4;
+        for (int e = threadIdx.x; e < NW4; e += 256) lla_cp_async16(pro_smem + 4 * e, wsrc + 4 * e);
     }
-    float* qr = pro_smem + (RK + 1) * DH + sl * DH;
-    if (active) {
+    const int k0 = (lane % KC) * 8, i0 = k0 < half ? k0 : k0 - half;  // the lane's k chunk and pairs
+    lla_cp_async_wait_all();
+    __syncthreads();
+    // A bound on every entry: entry (n, k) is x a + y b (k < d/2) or y a - x b (k >= d/2) with
+    // (x, y) = (q'_i, q'_{i+d/2}) and (a, b) = (w_n,i, w_n,i+d/2), so by Cauchy-Schwarz
+    // |entry| <= |(x, y)| |(a, b)|.  cw = the largest |(a, b)| over the head's rows.
+    float cw2 = 0.f;
+    for (int e = threadIdx.x; e < (RK + 1) * half; e += 256) {
+        const int n = e / half, i = e - n * half;
+        const float wa = pro_smem[n * DH + i], wb = pro_smem[n * DH + i + half];
+        cw2 = fmaxf(cw2, wa * wa + wb * wb);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cw2 = fmaxf(cw2, __shfl_xor_sync(0xffffffffu, cw2, o));
+    if (lane == 0) red[w] = cw2;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cw2 = fmaxf(cw2, red[j]);
+    const float cw = sqrtf(cw2);
+    const int part = h / C::HC, hc = h % C::HC, g = hc / C::HG, hg = hc % C::HG;
+    for (int j = 0; j < p.pro_spw; ++j) {
+        const int b = b_first + sl + sls * j;
+        if (b >= p.B) break;
         int qp = p.q_pos[b];
         if (qp < 0 || qp >= p.max_pos) {
             qp = qp < 0 ? 0 : p.max_pos - 1;
             if (h == 0 && wi == 0 && lane == 0) atomicOr(p.status, LLA_FLAG_POS_CLAMPED);
         }
+        // q' = scale * RoPE_qpos(q) on the lane's pairs i0 .. i0 + 8
         const float* qv = p.q + (size_t(b) * C::H + h) * DH;
-        for (int i = wi * 32 + lane; i < half; i += WPS * 32) {
-            const float c = p.rope_cos[size_t(qp) * half + i], sn = p.rope_sin[size_t(qp) * half + i];
-            const float lo = qv[i], hi = qv[i + half];
-            qr[i] = p.scale * (lo * c - hi * sn);
-            qr[i + half] = p.scale * (hi * c + lo * sn);
+        const float* cs = p.rope_cos + size_t(qp) * half + i0;
+        const float* sn = p.rope_sin + size_t(qp) * half + i0;
+        float x[8], y[8];
+        float pn = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float c = cs[u], sv = sn[u], lo = qv[i0 + u], hi = qv[i0 + u + half];
+            x[u] = p.scale * (lo * c - hi * sv);
+            y[u] = p.scale * (hi * c + lo * sv);
+            pn = fmaxf(pn, x[u] * x[u] + y[u] * y[u]);
         }
-    }
 #pragma unroll
-    for (int j = 0; j < WPT; ++j) {
-        const int e = threadIdx.x + 256 * j;
-        if (e < NW4) reinterpret_cast<float4*>(wt)[e] = wreg[j];
-    }
-    __syncthreads();
-    // element (n, k): k < d/2: q'_k w_k + q'_{k+d/2} w_{k+d/2};  k >= d/2: q'_{i+d/2} w_i - q'_i w_{i+d/2}
-    auto item = [&](int e, float* v) {
-        const int n = e / KC, k0 = (e - n * KC) * 8;
-        const int i0 = k0 < half ? k0 : k0 - half;
-        const float4* wl = reinterpret_cast<const float4*>(wt + size_t(n) * DH + i0);
-        const float4* wh = reinterpret_cast<const float4*>(wt + size_t(n) * DH + i0 + half);
-        const float4* ql = reinterpret_cast<const float4*>(qr + i0);
-        const float4* qh = reinterpret_cast<const float4*>(qr + i0 + half);
+        for (int o = KC / 2; o > 0; o >>= 1) pn = fmaxf(pn, __shfl_xor_sync(0xffffffffu, pn, o));  // every pair
+        // power-of-two scale keeping every entry below 2^15 (fp16 then keeps full precision;
+        // a power of two changes no rounding, and the scores are divided by it exactly)
+        const float bound = sqrtf(pn) * cw;
+        float scale = 1.f;
+        if (bound > 0.f && isfinite(bound)) {
+            int e2 = 0;
+            frexpf(bound, &e2);  // bound < 2^e2
+            scale = ldexpf(1.f, 15 - max(e2, -100));
+        }
+        uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
+        for (int e = wi * 32 + lane; e < NITEM; e += 32 * wps) {
+            const int n = e / KC;  // e % KC == lane % KC
+            const float4* wl = reinterpret_cast<const float4*>(pro_smem + n * DH + i0);
+            const float4* wh = reinterpret_cast<const float4*>(pro_smem + n * DH + i0 + half);
+            const float4 a0 = wl[0], a1 = wl[1], b0 = wh[0], b1 = wh[1];
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            __align__(16) __half hv[8];
 #pragma unroll
-        for (int u4 = 0; u4 < 2; ++u4) {
-            const float4 a = wl[u4], bb = wh[u4], x = ql[u4], y = qh[u4];
-            if (k0 < half) {
-                v[4 * u4 + 0] = x.x * a.x + y.x * bb.x;
-                v[4 * u4 + 1] = x.y * a.y + y.y * bb.y;
-                v[4 * u4 + 2] = x.z * a.z + y.z * bb.z;
-                v[4 * u4 + 3] = x.w * a.w + y.w * bb.w;
-            } else {
-                v[4 * u4 + 0] = y.x * a.x - x.x * bb.x;
-                v[4 * u4 + 1] = y.y * a.y - x.y * bb.y;
-                v[4 * u4 + 2] = y.z * a.z - x.z * bb.z;
-                v[4 * u4 + 3] = y.w * a.w - x.w * bb.w;
+            for (int u = 0; u < 8; ++u) {
+                const float v = k0 < half ? x[u] * av[u] + y[u] * bv[u] : y[u] * av[u] - x[u] * bv[u];
+                hv[u] = __float2half_rn(v * scale);
             }
+            const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
+            *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = *reinterpret_cast<const uint4*>(hv);
         }
-    };
-    // few items per lane: the values stay in registers (one pass over W);
-    // many: a max pass, then the values are recomputed for the write pass
-    constexpr int NPL = (NITEM + 32 * WPS - 1) / (32 * WPS);  // items per lane
-    constexpr bool KEEP = NPL <= 12;
-    const int e0 = wi * 32 + lane;
-    float keep[KEEP ? NPL : 1][8];
-    float mx = 0.f;
-#pragma unroll
-    for (int it = 0; it < NPL; ++it) {
-        const int e = e0 + 32 * WPS * it;
-        if (active && e < NITEM) {
-            float* v = keep[KEEP ? it : 0];
-            item(e, v);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) mx = fmaxf(mx, fabsf(v[u]));
-        }
+        if (hg == 0 && wi == 0)  // the group's padding rows
+            for (int e = lane; e < (C::NG - C::HG * (RK + 1)) * KC; e += 32) {
+                const int rowi = C::HG * (RK + 1) + e / KC, kk = (e % KC) * 8;
+                *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, kk, C::NG)) = make_uint4(0, 0, 0, 0);
+            }
+        if (wi == 0 && lane == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red[w] = mx;
-    __syncthreads();
-    if (!active) return;
-    for (int j = 0; j < WPS; ++j) mx = fmaxf(mx, red[sl * WPS + j]);
-    // power-of-two scale bringing the largest magnitude into [2^14, 2^15): fp16 keeps full precision
-    int e2 = 0;
-    float scale = 1.f;
-    if (mx > 0.f && isfinite(mx)) {
-        frexpf(mx, &e2);  // mx < 2^e2
-        scale = ldexpf(1.f, 15 - e2);
-    }
-    const int part = h / C::HC, hc = h % C::HC, g = hc / C::HG, hg = hc % C::HG;
-    uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
-#pragma unroll
-    for (int it = 0; it < NPL; ++it) {
-        const int e = e0 + 32 * WPS * it;
-        if (e >= NITEM) break;
-        float vv[8];
-        if (!KEEP) item(e, vv);
-        const float* v = KEEP ? keep[it] : vv;
-        const int n = e / KC, k0 = (e - n * KC) * 8;
-        const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
-        __align__(16) __half hv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) hv[u] = __float2half_rn(v[u] * scale);
-        *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = *reinterpret_cast<const uint4*>(hv);
-    }
-    if (hg == 0 && wi == 0)  // the group's padding rows
-        for (int e = lane; e < (C::NG - C::HG * (RK + 1)) * KC; e += 32) {
-            const int rowi = C::HG * (RK + 1) + e / KC, k0 = (e % KC) * 8;
-            *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = make_uint4(0, 0, 0, 0);
-        }
-    if (wi == 0 && lane == 0) p.inv_scale[size_t(b) * C::H + h] = kLog2e / scale;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -911,8 +882,6 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.lens = reinterpret_cast<int32_t*>(ws + L.off_lens);
     pp.inv_scale = reinterpret_cast<float*>(ws + L.off_isc);
     pp.mq = reinterpret_cast<uint8_t*>(ws + L.off_mq);
-    pp.records = reinterpret_cast<float*>(ws + L.off_rec);
-    pp.n_record_floats = (L.total - L.off_rec) / sizeof(float);
     pp.status = reinterpret_cast<uint32_t*>(ws);
     pp.B = B;
     pp.D = c->desc.D;
@@ -932,13 +901,22 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     pp.variant = c->desc.variant;
     pp.scale = call.scale;
     pp.smap = call.smap;
-    // split records start empty (l = 0); the combine skips them
-    LLA_CUDA_TRY(cudaMemsetAsync(pp.records, 0, pp.n_record_floats * sizeof(float), call.stream));
-    constexpr int pro_items = (C::RK + 1) * (C::DH / 8);
-    constexpr int pro_spc = pro_items >= 1024 ? 1 : pro_items >= 512 ? 2 : pro_items >= 256 ? 4 : 8;  // 8 / WPS
-    const size_t pro_smem = size_t(C::RK + 1 + pro_spc) * C::DH * sizeof(float);
+    // every record the combine reads is written by this call's decode kernel (a CTA writes all
+    // of its record set for each sequence it touches; the combine skips groups with no tiles)
+    // about four CTAs of eight warps per SM: many sequences run whole on one warp each (and a
+    // warp takes several in turn); few are spread over up to eight warps each
+    {
+        const long long tasks = (long long)B * C::H, target = 32LL * lla_num_sms();
+        pp.pro_wps = 1;
+        pp.pro_spw = 1;
+        if (tasks >= target) pp.pro_spw = int((tasks + target - 1) / target);
+        else
+            while (pp.pro_wps < 8 && tasks * pp.pro_wps < target) pp.pro_wps *= 2;
+    }
+    const int pro_per_cta = (8 / pp.pro_wps) * pp.pro_spw;
+    const size_t pro_smem = size_t(C::RK + 1) * C::DH * sizeof(float);
     LLA_CUDA_TRY(cudaFuncSetAttribute(tc_prologue_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pro_smem)));
-    tc_prologue_kernel<C><<<1 + C::H * ((B + pro_spc - 1) / pro_spc), 256, pro_smem, call.stream>>>(pp);
+    tc_prologue_kernel<C><<<1 + C::H * ((B + pro_per_cta - 1) / pro_per_cta), 256, pro_smem, call.stream>>>(pp);
     LLA_CUDA_TRY(cudaGetLastError());
 
     // Tensor map over the layer's latents: dims (row elems, head, token, sequence).  Per-head
@@ -983,7 +961,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     tp.P = pp.P;
     tp.lens = pp.lens;
     tp.inv_scale = pp.inv_scale;
-    tp.records = pp.records;
+    tp.records = reinterpret_cast<float*>(ws + L.off_rec);
     tp.status = pp.status;
     tp.B = B;
     tp.G = G;
@@ -1004,7 +982,7 @@ lla_status run_tc(const lla_decode_call& call, int num_ctas) {
     ranges.G = G;
     ranges.parts = C::PARTS;
     ranges.hc = C::HC;
-    return lla_combine_tc(call, pp.records, ranges);
+    return lla_combine_tc(call, tp.records, ranges);
 }
 
 using CfgRho21 = Cfg<128, 16, 32, 16>;

@@ -154,6 +154,22 @@ lla_status lla_full_decode(int H, float rope_base, const uint16_t* k_cache, cons
 // tail.
 __device__ __forceinline__ void lla_grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Asynchronous global -> shared copies of 4 or 16 bytes (no registers held while in flight);
+// lla_cp_async_wait_all() waits for every copy this thread issued.
+__device__ __forceinline__ void lla_cp_async4(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(uint32_t(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void lla_cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void lla_cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t lla_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                               bool pdl, Args... args) {
