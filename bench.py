@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.CONFIGS))
     ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--kernel-sample", type=int, default=8,
+                    help="time the decode kernel with CUDA events around every Nth call of the timed steps; "
+                         "the other calls launch as without events (programmatic dependent launch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
@@ -423,15 +426,19 @@ def run_ours(a, cfg):
         step()
     torch.cuda.synchronize()
 
-    # kernel events: one (begin, end) pair per decode call of the timed steps
-    ev_objs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(T * D)] for _ in range(a.steps)]
+    # kernel events: a (begin, end) pair around every kernel_sample-th decode call of the timed
+    # steps (an event between two kernels keeps the second from overlapping the first's tail,
+    # so the other calls launch as they do without events)
+    every = max(1, a.kernel_sample)
+    ev_objs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if k % every == 0
+                else None for k in range(T * D)] for _ in range(a.steps)]
     for row in ev_objs:
-        for e0, e1 in row:
-            e0.record()
-            e1.record()
+        for pair in row:
+            if pair is not None:
+                pair[0].record()
+                pair[1].record()
     torch.cuda.synchronize()
-    raw = [[(e0.cuda_event, e1.cuda_event) for e0, e1 in row] for row in ev_objs]
+    raw = [[(p[0].cuda_event, p[1].cuda_event) if p is not None else None for p in row] for row in ev_objs]
 
     if world > 1:
         dist.barrier()
@@ -446,7 +453,7 @@ def run_ours(a, cfg):
     if world > 1:
         dist.barrier()
     ms = g0.elapsed_time(g1)
-    kern_ms = [e0.elapsed_time(e1) for row in ev_objs for e0, e1 in row]
+    kern_ms = [p[0].elapsed_time(p[1]) for row in ev_objs for p in row if p is not None]
     ms_max = max_over_ranks(ms, dev)
     ctx_tokens_step = B * N * T * D
     value = job_value(ctx_tokens_step, a.steps, world, ms_max)
@@ -493,7 +500,9 @@ def run_ours(a, cfg):
                                **({"store": f"paged: {pages} pages of {lla.PAGE_TOKENS} tokens per sequence, "
                                             "shuffled over the pool"} if table is not None else {})),
                 "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
-                "roofline": roofline(cfg, kernel_name, kern_ms, a.workload),
+                "roofline": dict(roofline(cfg, kernel_name, kern_ms, a.workload),
+                                 timed_launches=f"{len(kern_ms)} of {a.steps * T * D}: every {every}th decode call "
+                                                "of the timed steps, bracketed by CUDA events on its stream"),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "clocks": clk.summary(),
                 "gpu_launches": a.steps * (T * D * LAUNCHES_PER_DECODE[kernel_name] + LAUNCHES_PER_ENCODE)}

@@ -30,8 +30,10 @@ constexpr int kThreads = 256;
 constexpr int kSeqPerCta = kThreads / 32;  // one warp per sequence
 constexpr int kMaxRowsPerLane = 8;         // output dimensions per lane: d <= 256
 
-// Row pitch of the staged W^V_up,t: odd, so rows i and i + 1 start in different banks.
-__host__ __device__ inline int w_pitch(int rv) { return rv | 1; }
+// Row pitch of the staged W^V_up,t.  r_v a multiple of 4: 4 (mod 32) words, so that eight
+// lanes reading 16 bytes each from eight consecutive rows cover the 32 banks once; otherwise
+// odd, so that rows i and i + 1 start in different banks.
+__host__ __device__ inline int w_pitch(int rv) { return rv % 4 == 0 ? (rv + 27) / 32 * 32 + 4 : rv | 1; }
 
 struct CombineParams {
     const float* partials;
@@ -103,8 +105,14 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
         r.total = total;
         r.groups = groups;
         const long long x0 = p.tc_P[b], x1 = x0 + tiles - 1;
-        r.g0 = ((x0 + 1) * groups - 1) / total;
-        const long long g1 = ((x1 + 1) * groups - 1) / total;
+        long long g1;
+        if ((x1 + 1) * groups < (1LL << 32)) {  // the usual sizes: 32-bit divisions
+            r.g0 = uint32_t((x0 + 1) * groups - 1) / uint32_t(total);
+            g1 = uint32_t((x1 + 1) * groups - 1) / uint32_t(total);
+        } else {
+            r.g0 = ((x0 + 1) * groups - 1) / total;
+            g1 = ((x1 + 1) * groups - 1) / total;
+        }
         r.n = int(4 * (g1 - r.g0 + 1));
     } else {
         r.hstride = p.H;
@@ -124,7 +132,7 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
 // A lane holds NC latent dimensions (a = lane + 32 c, c < NC, 32 NC >= r_v) and RPL output
 // rows (32 RPL >= the CTA's rows).  The warp's loads
 // go out in as few dependent rounds as the data allows: W (asynchronous copies into shared
-// memory) and mu before the wait for the decode kernel, then the record set's bounds, then every
+// memory) before the wait for the decode kernel, then the record set's bounds, then every
 // record's (m, l) together with the acc of the first kRC records; the merge and the projection
 // then run from registers and shared memory.
 template <int NC, int RPL>
@@ -137,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
     const int d = p.d, rv = p.r_v, pitch = w_pitch(rv);
     const int rows = d / gridDim.z;  // output dimensions of this CTA's slice (gridDim.z divides d)
     const int i0 = blockIdx.z * rows;
-    extern __shared__ float smem[];
+    extern __shared__ __align__(16) float smem[];
     float* Ws = smem;                         // [rows][pitch]: row r holds W^V_up,t[i0 + r][0..rv)
     float* abar = Ws + rows * pitch + warp * rv;  // [kSeqPerCta][rv]
 
@@ -165,14 +173,7 @@ __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
             }
         }
     }
-    // mu of this lane's output rows r = lane + 32 k
-    float muv[RPL];
-#pragma unroll
-    for (int k = 0; k < RPL; ++k) {
-        const int r = lane + 32 * k;
-        muv[k] = (active && r < rows) ? __ldg(p.mu_v + mu_off + i0 + r) : 0.f;
-    }
-    lla_grid_dependency_wait();  // W and mu are constants; the records come from the decode kernel
+    lla_grid_dependency_wait();  // W is a constant; the records come from the decode kernel
 
     const size_t bh = size_t(b) * p.H + h;
     float L = 0.f, w_self = 0.f;
@@ -300,16 +301,35 @@ __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
     }
     // out_i = abar . W^V_up,t[i] + (1 - w_self) mu^V_t[i] + w_self v_self[i] for i = i0 + r,
     // r = lane + 32 k; the rows of a lane keep independent accumulation chains
-    float acc[RPL];
+    float acc[RPL], muv[RPL];  // mu of the lane's rows: loaded under the projection's arithmetic
 #pragma unroll
-    for (int k = 0; k < RPL; ++k) acc[k] = 0.f;
+    for (int k = 0; k < RPL; ++k) {
+        acc[k] = 0.f;
+        muv[k] = lane + 32 * k < rows ? __ldg(p.mu_v + mu_off + i0 + lane + 32 * k) : 0.f;
+    }
     const float* wr = Ws + size_t(min(lane, rows - 1)) * pitch;
     const int nk = (rows + 31) / 32;
-    for (int a = 0; a < rv; ++a) {
-        const float x = abar[a];
+    if (rv % 4 == 0) {  // 16-byte reads of W rows and of abar (pitch and rv multiples of 4)
+#pragma unroll 2
+        for (int a = 0; a < rv; a += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(abar + a);
 #pragma unroll
-        for (int k = 0; k < RPL; ++k)
-            if (k < nk && lane + 32 * k < rows) acc[k] = fmaf(x, wr[size_t(32 * k) * pitch + a], acc[k]);
+            for (int k = 0; k < RPL; ++k)
+                if (k < nk && lane + 32 * k < rows) {
+                    const float4 w = *reinterpret_cast<const float4*>(wr + size_t(32 * k) * pitch + a);
+                    acc[k] = fmaf(x.x, w.x, acc[k]);
+                    acc[k] = fmaf(x.y, w.y, acc[k]);
+                    acc[k] = fmaf(x.z, w.z, acc[k]);
+                    acc[k] = fmaf(x.w, w.w, acc[k]);
+                }
+        }
+    } else {
+        for (int a = 0; a < rv; ++a) {
+            const float x = abar[a];
+#pragma unroll
+            for (int k = 0; k < RPL; ++k)
+                if (k < nk && lane + 32 * k < rows) acc[k] = fmaf(x, wr[size_t(32 * k) * pitch + a], acc[k]);
+        }
     }
 #pragma unroll
     for (int k = 0; k < RPL; ++k) {

@@ -735,6 +735,16 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         for (int e = threadIdx.x; e < NW4; e += 256) lla_cp_async16(pro_smem + 4 * e, wsrc + 4 * e);
     }
     const int k0 = (lane % KC) * 8, i0 = k0 < half ? k0 : k0 - half;  // the lane's k chunk and pairs
+    const bool q_vec = (reinterpret_cast<uintptr_t>(p.q) & 15) == 0;   // q rows are d floats apart
+    auto ld8 = [](float* v, const float* src, bool vec) {
+        if (vec) {
+            const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+            v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = src[u];
+        }
+    };
     lla_cp_async_wait_all();
     __syncthreads();
     // A bound on every entry: entry (n, k) is x a + y b (k < d/2) or y a - x b (k >= d/2) with
@@ -764,15 +774,17 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
         }
         // q' = scale * RoPE_qpos(q) on the lane's pairs i0 .. i0 + 8
         const float* qv = p.q + (size_t(b) * C::H + h) * DH;
-        const float* cs = p.rope_cos + size_t(qp) * half + i0;
-        const float* sn = p.rope_sin + size_t(qp) * half + i0;
+        float cv[8], sv[8], lo[8], hi[8];
+        ld8(cv, p.rope_cos + size_t(qp) * half + i0, true);
+        ld8(sv, p.rope_sin + size_t(qp) * half + i0, true);
+        ld8(lo, qv + i0, q_vec);
+        ld8(hi, qv + i0 + half, q_vec);
         float x[8], y[8];
         float pn = 0.f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const float c = cs[u], sv = sn[u], lo = qv[i0 + u], hi = qv[i0 + u + half];
-            x[u] = p.scale * (lo * c - hi * sv);
-            y[u] = p.scale * (hi * c + lo * sv);
+            x[u] = p.scale * (lo[u] * cv[u] - hi[u] * sv[u]);
+            y[u] = p.scale * (hi[u] * cv[u] + lo[u] * sv[u]);
             pn = fmaxf(pn, x[u] * x[u] + y[u] * y[u]);
         }
 #pragma unroll
@@ -786,6 +798,15 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
             frexpf(bound, &e2);  // bound < 2^e2
             scale = ldexpf(1.f, 15 - max(e2, -100));
         }
+        // the lane's entries are pa a + pb b: (pa, pb) = (x, y) for k < d/2, (y, -x) beyond;
+        // scaling by a power of two is exact
+        const bool upper = k0 >= half;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float xs = x[u] * scale, ys = y[u] * scale;
+            x[u] = upper ? ys : xs;
+            y[u] = upper ? -xs : ys;
+        }
         uint8_t* img = p.mq + (size_t(part) * p.B + b) * size_t(C::MQ_BYTES) + size_t(g) * C::MQ_GROUP_BYTES;
         for (int e = wi * 32 + lane; e < NITEM; e += 32 * wps) {
             const int n = e / KC;  // e % KC == lane % KC
@@ -794,12 +815,10 @@ __global__ void __launch_bounds__(256) tc_prologue_kernel(ProParams p) {
             const float4 a0 = wl[0], a1 = wl[1], b0 = wh[0], b1 = wh[1];
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            __align__(16) __half hv[8];
+            __align__(16) __half2 hv[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float v = k0 < half ? x[u] * av[u] + y[u] * bv[u] : y[u] * av[u] - x[u] * bv[u];
-                hv[u] = __float2half_rn(v * scale);
-            }
+            for (int u = 0; u < 8; u += 2)
+                hv[u / 2] = __floats2half2_rn(x[u] * av[u] + y[u] * bv[u], x[u + 1] * av[u + 1] + y[u + 1] * bv[u + 1]);
             const int rowi = n < RK ? hg * RK + n : C::HG * RK + hg;
             *reinterpret_cast<uint4*>(img + sm100::sw128_offset(rowi, k0, C::NG)) = *reinterpret_cast<const uint4*>(hv);
         }
