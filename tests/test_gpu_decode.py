@@ -225,6 +225,39 @@ def test_rows_past_the_context_may_hold_nan(variant, rk, rv):
     lib.close()
 
 
+@pytest.mark.parametrize("variant,rk,rv", [(0, 16, 32), (0, 96, 160), (1, 64, 128)])
+def test_stale_workspace_does_not_reach_the_output(variant, rk, rv):
+    """The workspace is not cleared between calls: every split record the combine reads is
+    written by the same call, and a CTA group whose share of the tiles is empty (a batch with
+    fewer tiles than groups) is skipped.  A workspace full of NaN bytes, then the same workspace
+    reused with other lengths, gives the oracle's outputs both times."""
+    B, N, D, T, H, d = 3, 300, 1, 2, 16, 128
+    tag = f"stale_ws/{variant}/{rk}"
+    cfg = dict(D=D, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0, mu_var=0.1)
+    codec = rounded_codec(syn.seeded_codec(cfg, tag))
+    head = () if variant == 1 else (H,)
+    cK = syn.round_bf16(syn.gaussian(tag + "/cK", (B, D, N) + head + (rk,)))
+    cV = syn.round_bf16(syn.gaussian(tag + "/cV", (B, D, N) + head + (rv,)))
+    q = syn.round_f32(syn.gaussian(tag + "/q", (B, H, d)))
+    lib = make_lib_codec(lla, dict(D=D, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0,
+                                   max_pos=N + 4), codec)
+    assert _tc_supported(lib, B, N)
+    store = torch.from_numpy(to_bf16_bits(np.concatenate([cK, cV], -1)).view(np.int16)).to(DEV)
+    qd = torch.from_numpy(np.ascontiguousarray(q, np.float32)).to(DEV)
+    ws = torch.full((lib.workspace_bytes(B, N),), 0xFF, dtype=torch.uint8, device=DEV)
+    scale = 1 / math.sqrt(d)
+    for loop, lens in ((1, [300, 1, 0]), (0, [129, 300, 5])):
+        ln = torch.tensor(lens, dtype=torch.int32, device=DEV)
+        out = torch.full((B, H, d), float("nan"), dtype=torch.float32, device=DEV)
+        lla.decode_attn(lib, store, B, N, 0, loop, qd, ln, ln, scale, out, ws, impl=lla.IMPL_TC)
+        torch.cuda.synchronize()
+        assert lla.workspace_flags(ws) == 0
+        got = out.cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all(), lens
+        assert_close(got, oracle_decode(codec, cfg, cK[:, 0], cV[:, 0], q, 0, loop, lens, lens, scale), f"lens {lens}")
+    lib.close()
+
+
 # ---------------------------------------------------------------------------------------------
 # range flags
 # ---------------------------------------------------------------------------------------------
