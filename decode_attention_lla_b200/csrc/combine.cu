@@ -158,17 +158,19 @@ __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
         mu_off = size_t(p.layer) * p.T * p.H * d + (size_t(p.loop) * p.H + h) * d;
     }
     {
-        // W is read in its own (coalesced) order; each element lands at its padded place
+        // W is read in its own (coalesced) order; each element (four of them when r_v is a multiple
+        // of 4: rows and pitch then keep 16-byte alignment) lands at its padded place
         const float* wg = p.w_up_v + w_off + size_t(i0) * rv;
-        const int nw = rows * rv;
-        int r = threadIdx.x / rv, a = threadIdx.x - (threadIdx.x / rv) * rv;
-        const int dr = kThreads / rv, da = kThreads - (kThreads / rv) * rv;
+        const int vec = rv % 4 == 0 ? 4 : 1, rw = rv / vec, nw = rows * rw;
+        int r = threadIdx.x / rw, a = threadIdx.x - (threadIdx.x / rw) * rw;
+        const int dr = kThreads / rw, da = kThreads - (kThreads / rw) * rw;
         for (int e = threadIdx.x; e < nw; e += kThreads) {
-            lla_cp_async4(Ws + size_t(r) * pitch + a, wg + e);
+            if (vec == 4) lla_cp_async16(Ws + r * pitch + 4 * a, wg + 4 * e);
+            else lla_cp_async4(Ws + r * pitch + a, wg + e);
             r += dr;
             a += da;
-            if (a >= rv) {
-                a -= rv;
+            if (a >= rw) {
+                a -= rw;
                 ++r;
             }
         }
@@ -309,7 +311,20 @@ __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
     }
     const float* wr = Ws + size_t(min(lane, rows - 1)) * pitch;
     const int nk = (rows + 31) / 32;
-    if (rv % 4 == 0) {  // 16-byte reads of W rows and of abar (pitch and rv multiples of 4)
+    if (RPL <= 4 && rv == 32 * NC && rows == 32 * RPL) {  // whole blocks: no guards, fixed offsets
+#pragma unroll 4
+        for (int a = 0; a < 32 * NC; a += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(abar + a);
+#pragma unroll
+            for (int k = 0; k < RPL; ++k) {
+                const float4 w = *reinterpret_cast<const float4*>(wr + 32 * k * pitch + a);
+                acc[k] = fmaf(x.x, w.x, acc[k]);
+                acc[k] = fmaf(x.y, w.y, acc[k]);
+                acc[k] = fmaf(x.z, w.z, acc[k]);
+                acc[k] = fmaf(x.w, w.w, acc[k]);
+            }
+        }
+    } else if (rv % 4 == 0) {  // 16-byte reads of W rows and of abar (pitch and rv multiples of 4)
 #pragma unroll 2
         for (int a = 0; a < rv; a += 4) {
             const float4 x = *reinterpret_cast<const float4*>(abar + a);
@@ -391,10 +406,12 @@ static lla_status launch_combine(const lla_decode_call& call, CombineParams& p) 
     while (ds.d_head % (64 * z) == 0 && ds.H * seq_ctas * z < 2 * lla_num_sms()) z *= 2;
     const size_t smem = (size_t(w_pitch(ds.r_v)) * (ds.d_head / z) + size_t(kSeqPerCta) * ds.r_v) * sizeof(float);
     void (*kernel)(CombineParams) = nullptr;
-    const bool rows4 = ds.d_head / z <= 128;
+    const int rows = ds.d_head / z;  // rows per lane: 2, 4 or 8 blocks of 32
     switch ((ds.r_v + 31) / 32) {
-#define LLA_COMBINE_CASE(nc) \
-    case nc: kernel = rows4 ? combine_kernel<nc, 4> : combine_kernel<nc, kMaxRowsPerLane>; break;
+#define LLA_COMBINE_CASE(nc)                                                                        \
+    case nc:                                                                                        \
+        kernel = rows <= 64 ? combine_kernel<nc, 2> : rows <= 128 ? combine_kernel<nc, 4> : combine_kernel<nc, 8>; \
+        break;
         LLA_COMBINE_CASE(1)
         LLA_COMBINE_CASE(2)
         LLA_COMBINE_CASE(3)
