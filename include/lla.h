@@ -150,6 +150,8 @@ size_t lla_decode_workspace_bytes(const lla_codec* codec, int batch, int max_tok
  *   out       device float32 [batch][H][d_head]
  *   workspace device, >= lla_decode_workspace_bytes(codec, batch, max_tokens),
  *             16-byte aligned; the library owns its contents during the call.
+ *             They need no initialisation and carry nothing from one call to
+ *             the next (only the status word is read afterwards).
  *   Concurrent calls must use distinct workspaces.
  */
 lla_status lla_decode_attn(const lla_codec* codec, const uint16_t* store, int batch,
