@@ -16,10 +16,11 @@
 //
 // One CTA per (head, 8 sequences, slice of output dimensions), one warp per sequence: the rows
 // of W^V_up,t of its slice are copied asynchronously into shared memory, read from global
-// memory in their own order (coalesced) and kept row-major with an odd row pitch, so that the
-// lanes of a warp (one output dimension each at a time) read distinct banks.  Small batches split d into 32-row
-// slices to fill the machine, and every CTA of a (head, sequence) then merges the records
-// itself (cheap next to the projection); large batches keep all d rows in one CTA.
+// memory in their own order (coalesced) and kept row-major at a padded pitch (w_pitch), so
+// that the lanes of a warp (one output dimension each) read distinct banks.  Small batches
+// split d into 32-row slices to fill the machine, and every CTA of a (head, sequence) then
+// merges the records itself (cheap next to the projection); large batches keep all d rows in
+// one CTA.
 #include <math.h>
 
 #include "lla_internal.cuh"
@@ -130,11 +131,10 @@ __device__ __forceinline__ RecordSet record_set(const CombineParams& p, int b, i
 
 // One warp per (sequence, head); the CTA's eight warps share the rows of W^V_up,t of one head.
 // A lane holds NC latent dimensions (a = lane + 32 c, c < NC, 32 NC >= r_v) and RPL output
-// rows (32 RPL >= the CTA's rows).  The warp's loads
-// go out in as few dependent rounds as the data allows: W (asynchronous copies into shared
-// memory) before the wait for the decode kernel, then the record set's bounds, then every
-// record's (m, l) together with the acc of the first kRC records; the merge and the projection
-// then run from registers and shared memory.
+// rows (32 RPL >= the CTA's rows).  The warp's loads go out in as few dependent rounds as the
+// data allows: W (asynchronous copies into shared memory) before the wait for the decode
+// kernel, then the record set's bounds, then every record's (m, l) together with the acc of the
+// first kRC records; the merge and the projection then run from registers and shared memory.
 template <int NC, int RPL>
 __global__ void __launch_bounds__(kThreads, 3) combine_kernel(CombineParams p) {
     constexpr int kRC = NC <= 2 ? 8 : 16 / NC >= 2 ? 16 / NC : 2;  // records whose acc a lane holds at once
