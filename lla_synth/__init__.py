@@ -99,31 +99,34 @@ def orthonormal_columns(name: str, S: int, r: int) -> np.ndarray:
     return q * np.where(np.diag(rr) < 0, -1.0, 1.0)[None, :]
 
 
-def seeded_codec(cfg: dict, tag: str = "codec") -> dict:
+def seeded_codec(cfg: dict, tag: str = "codec", layers=None) -> dict:
     """A seeded codec: stacked W_up orthonormal, W_down equal to that stack, mu ~ N(0, mu_var).
 
     Per-head (variant 0): w_down [D,H,S,r], w_up [D,H,T,d,r], mu [D,H,S] with S = T*d.
     LLA-2D (variant 1):   w_down [D,S2,r],  w_up [D,T,H,d,r], mu [D,S2] with S2 = T*H*d,
     the stack ordered (loop, head, d).
+    Every (layer, head, axis) slot draws from its own seed, so `layers` (default: all) may name
+    the layers to draw; the others are left at zero.
     """
     D, T, H, d = cfg["D"], cfg["T"], cfg["H"], cfg["d_head"]
     mu_var = cfg.get("mu_var", 0.1)
+    layers = range(D) if layers is None else layers
     out = {}
     for axis, r in (("k", cfg["r_k"]), ("v", cfg["r_v"])):
         if cfg["variant"] == 0:
             S = T * d
-            wd = np.empty((D, H, S, r))
-            mu = np.empty((D, H, S))
-            for l in range(D):
+            wd = np.zeros((D, H, S, r))
+            mu = np.zeros((D, H, S))
+            for l in layers:
                 for h in range(H):
                     wd[l, h] = orthonormal_columns(f"{tag}/{axis}/l{l}/h{h}/w", S, r)
                     mu[l, h] = gaussian(f"{tag}/{axis}/l{l}/h{h}/mu", S, mu_var)
             wu = wd.reshape(D, H, T, d, r).copy()
         else:
             S2 = T * H * d
-            wd = np.empty((D, S2, r))
-            mu = np.empty((D, S2))
-            for l in range(D):
+            wd = np.zeros((D, S2, r))
+            mu = np.zeros((D, S2))
+            for l in layers:
                 wd[l] = orthonormal_columns(f"{tag}/{axis}/l{l}/w", S2, r)
                 mu[l] = gaussian(f"{tag}/{axis}/l{l}/mu", S2, mu_var)
             wu = wd.reshape(D, T, H, d, r).copy()
@@ -134,11 +137,21 @@ def seeded_codec(cfg: dict, tag: str = "codec") -> dict:
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
-    """Round float64 values to bf16 (nearest-even) and return them as float64."""
-    f = np.ascontiguousarray(a, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+    """Round float64 values to bf16 (nearest-even, via float32) and return them as float64.
+
+    Infinities and NaNs pass through unchanged; for every other float32 bit pattern the
+    increment cannot carry out of 32 bits."""
+    f = np.array(a, dtype=np.float32)
+    u = f.view(np.uint32)
+    special = (u & np.uint32(0x7F800000)) == np.uint32(0x7F800000)
+    kept = u[special] if special.any() else None
+    inc = (u >> np.uint32(16)) & np.uint32(1)
+    inc += np.uint32(0x7FFF)
+    u += inc
+    u &= np.uint32(0xFFFF0000)
+    if kept is not None:
+        u[special] = kept
+    return f.astype(np.float64)
 
 
 def round_f32(a: np.ndarray) -> np.ndarray:

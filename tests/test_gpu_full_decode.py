@@ -16,26 +16,12 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 import decode_attention_lla_b200 as lla  # noqa: E402
 import lla_synth as syn  # noqa: E402
-from lla_testutil import assert_close, from_bf16_bits, to_bf16_bits  # noqa: E402
+import parity_cases as PC  # noqa: E402
+from lla_testutil import to_bf16_bits  # noqa: E402
 from oracle import lla_oracle as O  # noqa: E402
 
 DEV = "cuda"
 NAN_BF16 = 0x7FC0
-
-
-def _cache(tag, B, L, N, H, d, lens):
-    """bf16 bits of [B][L][N][H][d] rotated keys and values (the oracle's order), NaN past lens."""
-    K = syn.gaussian(tag + "/K", (B, L, N, H, d))
-    pos = np.arange(N, dtype=np.float64)[None, None, :, None]
-    half = d // 2
-    th = pos[..., None] * np.power(10000.0, -2.0 * np.arange(half) / d)  # [1,1,N,1,half]
-    c, s = np.cos(th), np.sin(th)
-    Kr = np.concatenate([K[..., :half] * c - K[..., half:] * s, K[..., half:] * c + K[..., :half] * s], -1)
-    kb, vb = to_bf16_bits(Kr), to_bf16_bits(syn.gaussian(tag + "/V", (B, L, N, H, d)))
-    for b, n in enumerate(lens):
-        kb[b, :, n:] = NAN_BF16
-        vb[b, :, n:] = NAN_BF16
-    return kb, vb
 
 
 def _run(kb, vb, layer, B, L, N, H, d, q, qpos, lens, scale, num_ctas=0):
@@ -53,23 +39,22 @@ def _run(kb, vb, layer, B, L, N, H, d, q, qpos, lens, scale, num_ctas=0):
     return out.cpu().numpy().astype(np.float64), lla.workspace_flags(ws)
 
 
-@pytest.mark.parametrize("c", [dict(B=3, L=1, N=520, H=16, lens=[520, 0, 129]),
-                               dict(B=4, L=2, N=300, H=3, lens=[1, 300, 255, 77]),
-                               dict(B=2, L=1, N=1, H=1, lens=[1, 0])])  # one cached token: out = v_0
-def test_full_decode_matches_oracle(c):
+@pytest.mark.parametrize("ci", range(len(PC.FULL_CACHE)))
+def test_full_decode_matches_oracle(ci):
+    """Queries aimed at a few cached keys (the last one included), so the scores decide the result."""
+    c, Kr, V, q, qpos, scale = PC.full_cache_inputs(ci)
     B, L, N, H, d = c["B"], c["L"], c["N"], c["H"], 128
-    tag = f"full/{B}/{H}"
-    kb, vb = _cache(tag, B, L, N, H, d, c["lens"])
-    q = syn.round_f32(syn.gaussian(tag + "/q", (B, H, d)))
-    qpos = [n + 3 for n in c["lens"]]
-    scale = 1 / math.sqrt(d)
+    kb, vb = to_bf16_bits(Kr), to_bf16_bits(V)
+    for b, n in enumerate(c["lens"]):
+        kb[b, :, n:] = NAN_BF16
+        vb[b, :, n:] = NAN_BF16
     layer = L - 1
-    ref = O.full_decode(q, from_bf16_bits(kb[:, layer]), from_bf16_bits(vb[:, layer]), c["lens"], qpos, scale,
-                        10000.0)
+    ref = O.full_decode(q, Kr[:, layer], V[:, layer], c["lens"], qpos, scale, PC.ROPE_BASE)
+    zero = np.zeros((H, d))
     for ctas in (0, 1, 7, 300):
         got, flags = _run(kb, vb, layer, B, L, N, H, d, q, qpos, c["lens"], scale, ctas)
         assert flags == 0
-        assert_close(got, ref, f"full decode ctas {ctas}")
+        PC.assert_decode_close(got, ref, zero, f"full decode ctas {ctas}")
         assert np.all(got[np.array(c["lens"]) == 0] == 0)
 
 
@@ -87,29 +72,35 @@ def test_full_decode_argument_errors():
 
 def test_full_decode_full_size_sampled():
     """The comparator at the bench's size and launch configuration: batch 32 x 4096 x 16 heads, one
-    (layer, loop) slice of a cache with a larger sequence stride, one persistent CTA per SM;
-    sampled sequences (one ragged) checked against the oracle."""
-    B, H, d, N = 32, 16, 128, 4096
-    cap = N + 1
+    (layer, loop) slice of a cache with a larger sequence stride, one persistent CTA per SM.  The
+    cache is filled on the device; the sampled sequences' rows (one ragged) are overwritten with
+    host-drawn keys and values, their queries aimed at a few cached keys, and they are checked
+    against the oracle."""
+    f = PC.full_cache_full_size_sample()
+    c = PC.FULL_CACHE_SIZE
+    B, H, d, cap, sample = c["B"], c["H"], c["d"], f["cap"], c["sample"]
     stride = 2 * cap * H * d  # two slices per sequence: the call reads the second
     g = torch.Generator(device=DEV)
     g.manual_seed(syn.sub_seed("full/fullsize"))
     K = torch.empty(B * stride, dtype=torch.bfloat16, device=DEV).normal_(generator=g)
     V = torch.empty(B * stride, dtype=torch.bfloat16, device=DEV).normal_(generator=g)
-    q = torch.empty(B, H, d, device=DEV).normal_(generator=g)
-    lens = torch.full((B,), N, dtype=torch.int32, device=DEV)
-    lens[17] = N - 333
+    for T, host in ((K, f["K"]), (V, f["V"])):
+        view = T.view(B, 2, H, cap, d)
+        for i, b in enumerate(sample):
+            view[b, 1] = torch.from_numpy(host[i]).to(device=DEV, dtype=torch.bfloat16)
+    q = torch.empty(B, H, d, device=DEV).normal_(generator=g) * 8.0
+    q[torch.tensor(sample, device=DEV)] = torch.from_numpy(f["q"].astype(np.float32)).to(DEV)
+    lens = torch.from_numpy(f["lens_all"]).to(DEV)
     qpos = lens + 1
     out = torch.full((B, H, d), float("nan"), device=DEV)
     ws = torch.empty(lla.full_decode_workspace_bytes(H, d, B), dtype=torch.uint8, device=DEV)
     off = cap * H * d
-    scale = 1 / math.sqrt(d)
     lla.full_decode_attn(H, d, 10000.0, K.data_ptr() + 2 * off, V.data_ptr() + 2 * off, stride, B, cap, q, qpos, lens,
-                         scale, out, ws)
+                         f["scale"], out, ws)
     torch.cuda.synchronize()
     assert lla.workspace_flags(ws) == 0
-    sample = [0, 17, 31]
-    kv = lambda T: T.view(B, 2, H, cap, d)[sample, 1].float().cpu().numpy().astype(np.float64).transpose(0, 2, 1, 3)
-    ref = O.full_decode(q[sample].cpu().numpy().astype(np.float64), kv(K), kv(V), lens[sample].cpu().numpy(),
-                        qpos[sample].cpu().numpy(), scale, 10000.0)
-    assert_close(out[sample].cpu().numpy().astype(np.float64), ref, "full size sampled")
+    ref = O.full_decode(f["q"], f["K"].transpose(0, 2, 1, 3), f["V"].transpose(0, 2, 1, 3), f["lens"], f["qpos"],
+                        f["scale"], PC.ROPE_BASE)
+    e = PC.assert_decode_close(out[sample].cpu().numpy().astype(np.float64), ref, np.zeros((H, d)),
+                               "full size sampled")
+    print(f"full cache, full size: rel_l2={e[0]:.3e} max_abs={e[2]:.3e}")

@@ -17,29 +17,21 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 import decode_attention_lla_b200 as lla  # noqa: E402
 import lla_synth as syn  # noqa: E402
-from lla_testutil import assert_close, make_lib_codec, oracle_decode, rounded_codec, to_bf16_bits  # noqa: E402
+import parity_cases as PC  # noqa: E402
+from lla_testutil import make_lib_codec, rounded_codec, to_bf16_bits  # noqa: E402
 
 DEV = "cuda"
 P = lla.PAGE_TOKENS
 NAN_BF16 = 0x7FC0
 
-CASES = [
-    dict(variant=0, D=2, T=4, H=16, d_head=128, r_k=16, r_v=32, B=3, max_pages=4, lens=[512, 130, 0]),
-    dict(variant=0, D=1, T=4, H=16, d_head=128, r_k=96, r_v=160, B=2, max_pages=3, lens=[300, 257]),
-    dict(variant=1, D=2, T=4, H=16, d_head=128, r_k=64, r_v=128, B=3, max_pages=4, lens=[400, 1, 384]),
-    dict(variant=0, D=1, T=2, H=3, d_head=32, r_k=8, r_v=24, B=2, max_pages=3, lens=[200, 75]),
-]
+CASES = PC.PAGED
 
 
-def _setup(c, tag):
-    cfg = dict(c, rope_base=10000.0, mu_var=0.1)
-    codec = rounded_codec(syn.seeded_codec(cfg, tag))
-    B, D, H, d, mp = c["B"], c["D"], c["H"], c["d_head"], c["max_pages"]
+def _setup(c, ci, tag):
+    s = PC.paged_set(ci, tag)
+    B, D, mp = c["B"], c["D"], c["max_pages"]
     N = mp * P
-    head = () if c["variant"] == 1 else (H,)
-    cK = syn.round_bf16(syn.gaussian(tag + "/cK", (B, D, N) + head + (c["r_k"],)))
-    cV = syn.round_bf16(syn.gaussian(tag + "/cV", (B, D, N) + head + (c["r_v"],)))
-    bits = to_bf16_bits(np.concatenate([cK, cV], -1))  # [B, D, N, (H,) row]
+    bits = s.bits  # [B, D, N, (H,) row]
     for b, n in enumerate(c["lens"]):
         bits[b, :, n:] = NAN_BF16
     # pool: every sequence's pages in a shuffled order, plus spare pages of NaN
@@ -50,10 +42,8 @@ def _setup(c, tag):
     for b in range(B):
         for pg in range(mp):
             pool[table[b, pg]] = bits[b, :, pg * P:(pg + 1) * P]
-    q = syn.round_f32(syn.gaussian(tag + "/q", (B, H, d)))
-    lib = make_lib_codec(lla, dict(D=D, T=c["T"], H=H, d_head=d, r_k=c["r_k"], r_v=c["r_v"], variant=c["variant"],
-                                   rope_base=10000.0, max_pos=N + 8), codec)
-    return cfg, codec, lib, bits, pool, table, num_pages, cK, cV, q
+    lib = make_lib_codec(lla, s.desc_kw(N + 8), s.codec)
+    return s, lib, bits, pool, table, num_pages
 
 
 def _t(a, dt=torch.float32):
@@ -91,50 +81,49 @@ def _impls(c):
 @pytest.mark.parametrize("ci", range(len(CASES)))
 def test_paged_decode_equals_contiguous_and_oracle(ci):
     c = CASES[ci]
-    cfg, codec, lib, bits, pool, table, num_pages, cK, cV, q = _setup(c, f"paged{ci}")
-    scale = 1 / math.sqrt(c["d_head"])
-    layer, loop = c["D"] - 1, 1
-    ref = oracle_decode(codec, cfg, cK[:, layer], cV[:, layer], q, layer, loop, c["lens"], c["lens"], scale)
+    s, lib, bits, pool, table, num_pages = _setup(c, ci, f"paged{ci}")
+    case = s.case(c["D"] - 1, 1)
+    ref = case.reference()
     for impl in _impls(c):
-        out_c, fc, out_p, fp = _decode_both(lib, c, bits, pool, table, num_pages, q, c["lens"], layer, loop, impl)
+        out_c, fc, out_p, fp = _decode_both(lib, c, bits, pool, table, num_pages, case.q, c["lens"], case.layer,
+                                            case.loop, impl)
         assert fc == 0 and fp == 0
         assert np.array_equal(out_c, out_p), f"impl {impl}: paged differs from contiguous"
-        assert_close(out_p.astype(np.float64), ref, f"paged impl {impl}")
+        PC.assert_decode_close(out_p.astype(np.float64), ref, case.mu_v(), f"paged impl {impl}")
     lib.close()
 
 
 def test_paged_decode_with_self_slot():
     c = CASES[0]
-    cfg, codec, lib, bits, pool, table, num_pages, cK, cV, q = _setup(c, "paged_self")
-    ks = syn.round_f32(syn.gaussian("paged_self/ks", q.shape))
-    vs = syn.round_f32(syn.gaussian("paged_self/vs", q.shape))
-    scale = 1 / math.sqrt(c["d_head"])
-    ref = oracle_decode(codec, cfg, cK[:, 0], cV[:, 0], q, 0, 2, c["lens"], c["lens"], scale, k_self=ks, v_self=vs)
+    s, lib, bits, pool, table, num_pages = _setup(c, 0, "paged_self")
+    case = s.case(0, 2, self_slot=True)
+    ref = case.reference()
     for impl in _impls(c):
-        out_c, _, out_p, _ = _decode_both(lib, c, bits, pool, table, num_pages, q, c["lens"], 0, 2, impl, ks, vs)
+        out_c, _, out_p, _ = _decode_both(lib, c, bits, pool, table, num_pages, case.q, c["lens"], 0, 2, impl,
+                                          case.k_self, case.v_self)
         assert np.array_equal(out_c, out_p)
-        assert_close(out_p.astype(np.float64), ref, f"paged self impl {impl}")
+        PC.assert_decode_close(out_p.astype(np.float64), ref, case.mu_v(), f"paged self impl {impl}")
     lib.close()
 
 
 def test_invalid_page_cuts_the_sequence_and_is_flagged():
     c = CASES[0]
-    cfg, codec, lib, bits, pool, table, num_pages, cK, cV, q = _setup(c, "paged_bad")
+    s, lib, bits, pool, table, num_pages = _setup(c, 0, "paged_bad")
     bad = table.copy()
     bad[0, 2] = num_pages + 5  # sequence 0 (512 tokens) loses pages 2 and 3: 256 tokens remain
+    cut = list(c["lens"])
+    cut[0] = 2 * P
+    case = s.case(1, 0, lens=cut, qpos=c["lens"])
     for impl in _impls(c):
         B, mp = c["B"], c["max_pages"]
         ln = torch.tensor(c["lens"], dtype=torch.int32, device=DEV)
         ws = torch.empty(lib.workspace_bytes(B, mp * P), dtype=torch.uint8, device=DEV)
         out = torch.empty(B, 16, 128, device=DEV)
         lla.decode_attn_paged(lib, _t(pool.view(np.int16), torch.int16), num_pages, _t(bad, torch.int32), mp, B, 1, 0,
-                              _t(q), ln, ln, 1 / math.sqrt(128), out, ws, impl=impl)
+                              _t(case.q), ln, ln, case.scale, out, ws, impl=impl)
         torch.cuda.synchronize()
         assert lla.workspace_flags(ws) & lla.FLAG_PAGE_INVALID
-        cut = list(c["lens"])
-        cut[0] = 2 * P
-        ref = oracle_decode(codec, cfg, cK[:, 1], cV[:, 1], q, 1, 0, cut, c["lens"], 1 / math.sqrt(128))
-        assert_close(out.cpu().numpy().astype(np.float64), ref, f"cut impl {impl}")
+        PC.assert_decode_close(out.cpu().numpy().astype(np.float64), case.reference(), case.mu_v(), f"cut impl {impl}")
     lib.close()
 
 

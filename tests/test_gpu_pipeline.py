@@ -4,7 +4,8 @@ reconstruction, softmax attention], on the same seeded stacks and codec.
 
 The oracle consumes the latents rounded to bf16, as the store holds them; the GPU encode rounds
 to nearest-even too, so the two latent sets agree to within an ulp and the outputs within the
-acceptance bar.  Also: repeated decode calls on the same inputs are bit-identical.
+acceptance bar (on the output and on out - mu^V_t; queries aimed at a few cached keys, so the
+score path is exercised).  Also: repeated decode calls on the same inputs are bit-identical.
 """
 
 import math
@@ -17,8 +18,8 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 import decode_attention_lla_b200 as lla  # noqa: E402
 import lla_synth as syn  # noqa: E402
-from oracle import lla_oracle as O  # noqa: E402
-from lla_testutil import assert_close, make_lib_codec, oracle_decode, rounded_codec, to_bf16_bits  # noqa: E402
+import parity_cases as PC  # noqa: E402
+from lla_testutil import make_lib_codec, rounded_codec, to_bf16_bits  # noqa: E402
 
 DEV = "cuda"
 
@@ -29,65 +30,31 @@ SHAPES = [  # (variant, r_k, r_v): the three shapes the tensor-core kernels cove
 ]
 
 
-def _setup(variant, rk, rv, tag, B=2, N=300, T=4, H=16, d=128):
-    cfg = dict(D=1, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0, mu_var=0.1)
-    codec = rounded_codec(syn.seeded_codec(cfg, tag))
-    lib = make_lib_codec(lla, dict(D=1, T=T, H=H, d_head=d, r_k=rk, r_v=rv, variant=variant, rope_base=10000.0,
-                                   max_pos=N + 8), codec)
-    S = T * d if variant == 0 else T * H * d
-    n = B * N
-    if variant == 0:
-        x = np.empty((n, 1, H, 2, S))
-        for h in range(H):
-            for a in range(2):
-                x[:, 0, h, a] = syn.smooth_stacks(f"{tag}/x/{h}/{a}", n, T, d, 8, 1e-2,
-                                                  codec[f"mu_{'kv'[a]}"][0, h], basis_name=f"{tag}/b/{h}/{a}")
-    else:
-        x = np.empty((n, 1, 2, S))
-        for a in range(2):
-            x[:, 0, a] = syn.smooth_stacks(f"{tag}/x/{a}", n, T, H * d, 8, 1e-2, codec[f"mu_{'kv'[a]}"][0],
-                                           basis_name=f"{tag}/b/{a}")
-    x = syn.round_bf16(x)
-    return cfg, codec, lib, x, S
-
-
 @pytest.mark.parametrize("shape", SHAPES)
 def test_encode_then_decode_matches_oracle(shape):
+    """Queries aimed at a few cached keys of the oracle's latents, one decode call per loop."""
     variant, rk, rv = shape
-    B, N, H, d, T = 2, 300, 16, 128, 4
-    lens = [300, 171]
-    tag = f"pipe/{variant}/{rk}"
-    cfg, codec, lib, x, S = _setup(variant, rk, rv, tag, B, N, T, H, d)
+    H, d, T = 16, 128, 4
+    B, N, lens = PC.PIPE_B, PC.PIPE_N, PC.PIPE_LENS
+    x, lat = PC.pipeline_inputs(variant, rk, rv, T, H, d)
+    lib = make_lib_codec(lla, lat.desc_kw(N + 8), lat.codec)
     # GPU: every (sequence, token) stack encoded into its slot, then one decode call per loop
     seq = np.repeat(np.arange(B), N).astype(np.int32)
     tok = np.tile(np.arange(N), B).astype(np.int32)
     store = torch.zeros(lla.store_bytes(lib.desc, B, N) // 2, dtype=torch.int16, device=DEV)
     xd = torch.from_numpy(to_bf16_bits(x).view(np.int16)).to(DEV)
     lla.encode(lib, xd, B * N, 0, 1, torch.from_numpy(seq).to(DEV), torch.from_numpy(tok).to(DEV), store, B, N)
-    q = syn.round_f32(syn.gaussian(tag + "/q", (T, B, H, d)))
     ln = torch.tensor(lens, dtype=torch.int32, device=DEV)
     ws = torch.empty(lib.workspace_bytes(B, N), dtype=torch.uint8, device=DEV)
-    scale = 1 / math.sqrt(d)
-    # oracle: encode [LLA §3 eq. (2)], the store's bf16 rounding, decode
-    if variant == 0:
-        cK = np.empty((B * N, H, rk))
-        cV = np.empty((B * N, H, rv))
-        for h in range(H):
-            cK[:, h] = O.encode(x[:, 0, h, 0], codec["mu_k"][0, h], codec["w_down_k"][0, h])
-            cV[:, h] = O.encode(x[:, 0, h, 1], codec["mu_v"][0, h], codec["w_down_v"][0, h])
-        cK, cV = cK.reshape(B, N, H, rk), cV.reshape(B, N, H, rv)
-    else:
-        cK = O.encode(x[:, 0, 0], codec["mu_k"][0], codec["w_down_k"][0]).reshape(B, N, rk)
-        cV = O.encode(x[:, 0, 1], codec["mu_v"][0], codec["w_down_v"][0]).reshape(B, N, rv)
-    cK, cV = syn.round_bf16(cK), syn.round_bf16(cV)
+    # oracle: encode [LLA §3 eq. (2)] (the store's bf16 rounding included), then decode
     for t in range(T):
+        case = lat.case(0, t)
         out = torch.full((B, H, d), float("nan"), device=DEV)
-        qd = torch.from_numpy(q[t].astype(np.float32)).to(DEV)
-        lla.decode_attn(lib, store, B, N, 0, t, qd, ln, ln, scale, out, ws, impl=lla.IMPL_TC)
+        qd = torch.from_numpy(case.q.astype(np.float32)).to(DEV)
+        lla.decode_attn(lib, store, B, N, 0, t, qd, ln, ln, case.scale, out, ws, impl=lla.IMPL_TC)
         torch.cuda.synchronize()
         assert lla.workspace_flags(ws) == 0
-        ref = oracle_decode(codec, cfg, cK, cV, q[t], 0, t, lens, lens, scale)
-        assert_close(out.cpu().numpy().astype(np.float64), ref, f"loop {t}")
+        PC.assert_decode_close(out.cpu().numpy().astype(np.float64), case.reference(), case.mu_v(), f"loop {t}")
     lib.close()
 
 

@@ -17,16 +17,12 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 import decode_attention_lla_b200 as lla  # noqa: E402
 import lla_synth as syn  # noqa: E402
+import parity_cases as PC  # noqa: E402
 from lla_testutil import assert_close, make_lib_codec, oracle_decode, rounded_codec, to_bf16_bits  # noqa: E402
 
 DEV = "cuda"
 
-CASES = [
-    dict(variant=0, D=1, T=4, H=16, d_head=128, r_k=16, r_v=32, B=4, N=300, lens=[300, 0, 129, 77]),
-    dict(variant=0, D=1, T=4, H=16, d_head=128, r_k=96, r_v=160, B=3, N=260, lens=[260, 1, 128]),
-    dict(variant=1, D=1, T=4, H=16, d_head=128, r_k=64, r_v=128, B=3, N=400, lens=[400, 0, 131]),
-    dict(variant=0, D=2, T=2, H=3, d_head=32, r_k=8, r_v=24, B=3, N=90, lens=[90, 0, 33]),
-]
+CASES = PC.SELF
 
 
 def _case(c, tag):
@@ -62,21 +58,24 @@ def _tc_ok(c):
 
 @pytest.mark.parametrize("ci", range(len(CASES)))
 def test_self_slot_matches_oracle(ci):
+    """Queries aimed at a few cached keys (the self slot's logit is scale * <q, k_self>)."""
     c = CASES[ci]
-    cfg, codec, lib, bits, cK, cV, q, ks, vs = _case(c, f"self{ci}")
+    s = PC.self_set(ci)
+    lib = make_lib_codec(lla, s.desc_kw(c["N"] + 8), s.codec)
+    bits = s.bits
     B, N = c["B"], c["N"]
-    scale = 1 / math.sqrt(c["d_head"])
     impls = [lla.IMPL_SIMT] + ([lla.IMPL_TC] if _tc_ok(c) else [])
-    for layer, loop in ((0, 1), (c["D"] - 1, c["T"] - 1)):
-        ref = oracle_decode(codec, cfg, cK[:, layer], cV[:, layer], q, layer, loop, c["lens"], c["lens"], scale,
-                            k_self=ks, v_self=vs)
+    for layer, loop in PC.self_calls(ci):
+        case = s.case(layer, loop, self_slot=True)
+        ref = case.reference()
         for impl in impls:
-            got, flags = _run_self(lib, bits, B, N, layer, loop, q, c["lens"], ks, vs, scale, impl)
+            got, flags = _run_self(lib, bits, B, N, layer, loop, case.q, case.lens, case.k_self, case.v_self,
+                                   case.scale, impl)
             assert flags == 0
-            assert_close(got, ref, f"self slot impl {impl} layer {layer} loop {loop}")
+            PC.assert_decode_close(got, ref, case.mu_v(), f"self slot impl {impl} layer {layer} loop {loop}")
             # a sequence with no cached token attends to the self slot alone
             empty = np.array(c["lens"]) == 0
-            assert np.abs(got[empty] - vs[empty]).max(initial=0.0) < 1e-6
+            assert np.abs(got[empty] - case.v_self[empty]).max(initial=0.0) < 1e-6
     lib.close()
 
 
