@@ -13,7 +13,9 @@
 // library, for the life of the process.  Host code may not use the array's
 // name as a device address: on the host it names a stand-in object.  The
 // device address is looked up once per device with cudaGetSymbolAddress,
-// with that device current, and cached.
+// with that device current, and cached: after cudaDeviceReset on a device that has served a call
+// the cached address is stale, so the entry point does not support that reset (the process must
+// not call this entry point on that device again).
 #include <mutex>
 
 #include "lla_internal.cuh"
@@ -62,7 +64,10 @@ extern "C" lla_status lla_decode_attn_noalloc(const lla_codec* c, const uint16_t
     if (!store || !q || !q_pos || !seq_lens || !out) return LLA_ERR_INVALID_ARG;
     if (!aligned(store, 16) || !aligned(q, 16) || !aligned(out, 16) || !aligned(q_pos, 4) || !aligned(seq_lens, 4))
         return LLA_ERR_ALIGNMENT;
-    if (lla_simt_workspace_bytes(c, batch, max_tokens) > kScratchBytes) return LLA_ERR_WORKSPACE;
+    // The call always runs at the automatic split count, so that is what must fit (the general
+    // workspace size also reserves room for explicit split overrides, which this entry point
+    // never takes).
+    if (lla_simt_auto_workspace_bytes(c, batch, max_tokens) > kScratchBytes) return LLA_ERR_WORKSPACE;
 
     void* scratch = nullptr;
     const lla_status st = scratch_address(&scratch);

@@ -189,6 +189,15 @@ size_t lla_simt_workspace_bytes(const lla_codec* c, int batch, int max_tokens) {
     return sizeof(lla_ws_header) + size_t(batch) * splits * H * lla_partial_floats(c->desc.r_v) * sizeof(float);
 }
 
+size_t lla_simt_auto_workspace_bytes(const lla_codec* c, int batch, int max_tokens) {
+    // exactly what lla_decode_simt(call, 0) checks against: the automatic split count, clamped to
+    // the tile count as the launch clamps it
+    const int tiles = (max_tokens + kTile - 1) / kTile;
+    int splits = simt_splits(batch, c->desc.H, max_tokens);
+    if (splits > tiles) splits = tiles > 0 ? tiles : 1;
+    return sizeof(lla_ws_header) + size_t(batch) * splits * c->desc.H * lla_partial_floats(c->desc.r_v) * sizeof(float);
+}
+
 lla_status lla_decode_simt(const lla_decode_call& call, int splits_override) {
     const lla_codec* c = call.codec;
     const lla_codec_desc& ds = c->desc;

@@ -107,6 +107,8 @@ __host__ __device__ inline size_t lla_partial_floats(int r_v) { return size_t(r_
 
 // ---- host-side entry points implemented in the .cu files ------------------
 size_t lla_simt_workspace_bytes(const lla_codec* c, int batch, int max_tokens);
+// scratch of the CUDA-core kernel at its automatic split count (no explicit split override)
+size_t lla_simt_auto_workspace_bytes(const lla_codec* c, int batch, int max_tokens);
 lla_status lla_decode_simt(const lla_decode_call& call, int splits_override);
 size_t lla_tc_workspace_bytes(const lla_codec* c, int batch, int max_tokens);
 bool lla_tc_supported(const lla_codec* c);

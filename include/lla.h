@@ -351,17 +351,27 @@ lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* str
  *   their scratch in an 8 MiB array compiled into the library, which every
  *   GPU that loads the library holds until the process exits.  It calls no
  *   allocator of any kind.
- *   Limit: shapes whose workspace (lla_decode_workspace_bytes of the
- *   CUDA-core kernel: split records of batch x H x (r_v + 2) floats per
- *   split) exceeds 8 MiB are rejected with LLA_ERR_WORKSPACE before anything
- *   is launched.  The per-head workload with batch 768, H 16, r_v 32 needs
- *   about 1.7 MiB.
+ *   Limit: the scratch of one call is a 256-byte header plus the split records,
+ *   batch x splits x H x (r_v + 2) floats, where splits is the automatic
+ *   split count: ceil(4 x SMs / (batch x H)), at least 1 and at most
+ *   ceil(max_tokens / 128).  A call whose scratch exceeds 8 MiB is rejected
+ *   with LLA_ERR_WORKSPACE before anything is launched.  Once batch x H
+ *   reaches 4 x SMs (592 on a 148-SM B200) splits is 1, so with H 16 and
+ *   r_v 32 (2176 bytes per sequence) batches up to 3854 fit; the per-head
+ *   workload with batch 768 needs about 1.6 MiB.
  *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.  cudaDeviceReset on a device after a call here leaves the
+ *   cached address stale: this entry point must not be used on that device
+ *   again in the same process.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: the status word is cleared at the start of each call, the
  *   split records are rewritten.  Calls that overlap on the GPU (different
  *   streams, or different host threads without ordering) race on it.
+ *   The status word is not readable by the caller (the array has no address
+ *   the caller can pass to lla_workspace_flags): a seq_len above max_tokens
+ *   or a position outside [0, max_pos) is clamped as in lla_decode_attn, but
+ *   silently.  Callers that need the flags use lla_decode_attn.
  *   Arguments and results are those of lla_decode_attn without the
  *   workspace.
  */
