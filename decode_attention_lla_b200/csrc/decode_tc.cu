@@ -208,14 +208,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
     uint64_t* mq_empty = mq_full + 1;
     uint64_t* tm_full = mq_full + 2;          // [NBUF]
     uint64_t* tm_empty = tm_full + C::NBUF;  // [NBUF]
-    uint64_t* st_full = tm_empty + C::NBUF;  // [NST]
-    uint64_t* st_empty = st_full + C::NST;
+    // Round r of stage slot s lands on barrier st_full[r % 4][s].  Compute warps drift apart by
+    // up to NBUF head groups (a warp can only start a group once every warp has released the
+    // group NBUF before it), which can exceed a ring round: a parity wait on one barrier per
+    // slot could then match an earlier round of the slot.  With four barriers per slot a wait
+    // could only alias a round four rounds back, which every consumer has long released.
+    uint64_t* st_full = tm_empty + C::NBUF;  // [4][NST]
+    uint64_t* st_empty = st_full + 4 * C::NST;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(st_empty + C::NST);
-    // issued[s] = number of loads the producer has issued into stage slot s.  Consumer warps
-    // drift apart by more than the ring depth, so a parity wait alone could match the
-    // previous round of a slot; a consumer first waits until its round has been issued.
-    volatile uint32_t* issued = tmem_holder + 1;
-    if (threadIdx.x < C::NST) issued[threadIdx.x] = 0;
+    static_assert((4 + 2 * C::NBUF + 5 * C::NST) * 8 + 16 <= C::BAR_BYTES, "barrier area");
+    static_assert(C::NBUF * (C::STAGES_PER_TILE / C::GPC) <= 4 * C::NST, "stage rounds a wait can be ahead");
+    auto st_full_bar = [&](uint32_t slot, uint32_t round) { return st_full + (round & 3) * C::NST + slot; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -227,10 +230,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
             mbar_init(tm_full + i, 1);
             mbar_init(tm_empty + i, C::NCW);
         }
-        for (int i = 0; i < C::NST; ++i) {
-            mbar_init(st_full + i, 1);
-            mbar_init(st_empty + i, C::ST_CONSUMERS);
-        }
+        for (int i = 0; i < 4 * C::NST; ++i) mbar_init(st_full + i, 1);
+        for (int i = 0; i < C::NST; ++i) mbar_init(st_empty + i, C::ST_CONSUMERS);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -275,55 +276,65 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 6);
     };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ latent stage producer
-        if (elect_one()) {
-            prefetch_tensormap(&lat_map);
-            const uint64_t pol_stream = policy_evict_first();
-            uint32_t stage_k = 0;
-            bool ok = true;
-            for (; wk.valid() && ok; wk.next()) {
-                if (!C::PHI_WARP && !(ok = phi_mq_step())) break;
-                for (int hl = 0; hl < C::HC && ok; ++hl) {
-                    const int h = wk.p * C::HC + hl;
-                    for (int ch = 0; ch < C::CHUNKS; ++ch) {
-                        const uint32_t slot = stage_k % C::NST, round = stage_k / C::NST;
-                        if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
-                            break;
-                        mbar_expect_tx(st_full + slot, C::STAGE_BYTES);
-                        uint8_t* dst = stage_s + size_t(slot) * C::STAGE_BYTES;
-                        int tok, outer;
-                        tile_coords(p, wk.b, wk.t, tok, outer);
-                        tok += ch * C::TOKS;
-                        if constexpr (C::WIDE) {
-                            tma_load_4d(dst, &maps.m[0], 0, h, tok, outer, st_full + slot, pol_stream);
-                            tma_load_4d(dst + C::K0_BYTES, &maps.m[1], 64, h, tok, outer, st_full + slot, pol_stream);
-                            tma_load_4d(dst + C::V_OFF, &maps.m[2], C::RK, h, tok, outer, st_full + slot, pol_stream);
-                        } else {
-                            tma_load_4d(dst, &lat_map, 0, h, tok, outer, st_full + slot, pol_stream);
-                        }
-                        __threadfence_block();  // the armed barrier phase precedes the published round
-                        issued[slot] = round + 1;
-                        ++stage_k;
+    // Latent stages of the CTA's walk, in ring order.  With narrow rows the M_q/Phi warp issues
+    // the stages of odd heads and warp 0 those of even heads: one issuing thread shares its
+    // scheduler with four compute warps, and the loads of a tile went out measurably faster from
+    // two (about 4% per call).  With wide rows warp 0 issues every stage and the M_q/Phi loads.
+    auto produce = [&](int parity_sel, bool with_phi) {
+        prefetch_tensormap(&lat_map);
+        if (C::WIDE) {
+            prefetch_tensormap(&maps.m[1]);
+            prefetch_tensormap(&maps.m[2]);
+        }
+        const uint64_t pol_stream = policy_evict_first();
+        uint32_t stage_k = 0;
+        bool ok = true;
+        for (; wk.valid() && ok; wk.next()) {
+            if (with_phi && !(ok = phi_mq_step())) break;
+            int tok0, outer;
+            tile_coords(p, wk.b, wk.t, tok0, outer);
+            for (int hl = 0; hl < C::HC && ok; ++hl) {
+                if (parity_sel >= 0 && (hl & 1) != parity_sel) {
+                    stage_k += C::CHUNKS;  // the other producer's head
+                    continue;
+                }
+                const int h = wk.p * C::HC + hl;
+                for (int ch = 0; ch < C::CHUNKS; ++ch) {
+                    const uint32_t slot = stage_k % C::NST, round = stage_k / C::NST;
+                    if (round > 0 && !(ok = mbar_wait(st_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 3)))
+                        break;
+                    uint64_t* bar = st_full_bar(slot, round);
+                    mbar_expect_tx(bar, C::STAGE_BYTES);
+                    uint8_t* dst = stage_s + size_t(slot) * C::STAGE_BYTES;
+                    const int tok = tok0 + ch * C::TOKS;
+                    if constexpr (C::WIDE) {
+                        tma_load_4d(dst, &maps.m[0], 0, h, tok, outer, bar, pol_stream);
+                        tma_load_4d(dst + C::K0_BYTES, &maps.m[1], 64, h, tok, outer, bar, pol_stream);
+                        tma_load_4d(dst + C::V_OFF, &maps.m[2], C::RK, h, tok, outer, bar, pol_stream);
+                    } else {
+                        tma_load_4d(dst, &lat_map, 0, h, tok, outer, bar, pol_stream);
                     }
+                    ++stage_k;
                 }
             }
-            // No copy may still be in flight when the CTA exits.
-            for (uint32_t s = 0; s < C::NST && s < stage_k; ++s) {
-                const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last issue into slot s
-                mbar_wait(st_full + s, (last / C::NST) & 1, p.status, kFlagTimeout, 4);
-            }
-            if (!C::PHI_WARP) phi_mq_drain();
         }
+        // No copy this thread issued may still be in flight when the CTA exits.
+        for (uint32_t s = 0; s < C::NST && s < stage_k; ++s) {
+            const uint32_t last = stage_k - 1 - ((stage_k - 1 - s) % C::NST);  // last round of slot s
+            if (parity_sel >= 0 && ((last % C::STAGES_PER_TILE) / C::CHUNKS & 1) != uint32_t(parity_sel)) continue;
+            mbar_wait(st_full_bar(s, last / C::NST), (last / C::NST >> 2) & 1, p.status, kFlagTimeout, 4);
+        }
+        if (with_phi) phi_mq_drain();
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ latent stage producer
+        if (elect_one()) produce(C::PHI_WARP ? 0 : -1, !C::PHI_WARP);
     } else if (C::PHI_WARP && warp == 2) {
-        // ------------------------------------------------------------ M_q and Phi producer
-        // (its own warp, so the next tile's Phi goes out as soon as its buffer is free rather
-        // than behind the current tile's latent stages)
-        if (elect_one()) {
-            bool ok = true;
-            for (; wk.valid() && ok; wk.next()) ok = phi_mq_step();
-            phi_mq_drain();
-        }
+        // ------------------------------------------------------------ M_q, Phi and odd-head stages
+        // (the next tile's Phi goes out as soon as its buffer is free rather than behind the
+        // current tile's latent stages)
+        if (elect_one()) produce(1, true);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
@@ -402,10 +413,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
 
         auto wait_stage = [&](uint32_t slot, uint32_t round) {
             bool w_ok = true;
-            if (lane == 0) {
-                w_ok = ok && wait_issued(issued + slot, round + 1, p.status, kFlagTimeout, 14);
-                w_ok = w_ok && mbar_wait(st_full + slot, round & 1, p.status, kFlagTimeout, 13);
-            }
+            if (lane == 0) w_ok = ok && mbar_wait(st_full_bar(slot, round), (round >> 2) & 1, p.status, kFlagTimeout, 13);
             ok = __shfl_sync(0xffffffffu, w_ok, 0) && ok;
             __syncwarp();  // lane 0's barrier acquire covers the whole warp's reads
         };
