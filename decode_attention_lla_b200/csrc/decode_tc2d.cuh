@@ -61,8 +61,7 @@ struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
     static_assert(VCOL + 2 * VN <= TMEM_COLS, "TMEM columns");
     static_assert(NV >= 4, "c^V ring");
     static_assert(SMEM <= kSmemLimit, "shared memory");
-    static_assert((6 + 2 * NBUF + 6 + 2 * NK + 2 * NV) * 8 + 256 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
-    static_assert(1 + NK + NV <= 64, "issue counters");
+    static_assert((6 + 2 * NBUF + 6 + 5 * NK + 5 * NV) * 8 + 16 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
 };
 
 // Wait for the last phase of each of `ns` ring barriers after `count` uses in ring order.
@@ -71,6 +70,15 @@ __device__ __forceinline__ void wait_last_phases(uint64_t* bars, uint32_t ns, ui
     for (uint32_t s = 0; s < ns && s < count; ++s) {
         const uint32_t last = count - 1 - ((count - 1 - s) % ns);
         mbar_wait(bars + s, (last / ns) & 1, status, kFlagTimeout, site);
+    }
+}
+
+// The same for a ring whose round r of slot s lands on bars[r % 4][s] (four sets of ns).
+__device__ __forceinline__ void wait_last_phases4(uint64_t* bars, uint32_t ns, uint32_t count, uint32_t* status,
+                                                  uint32_t site) {
+    for (uint32_t s = 0; s < ns && s < count; ++s) {
+        const uint32_t last = (count - 1 - ((count - 1 - s) % ns)) / ns;  // last round of slot s
+        mbar_wait(bars + (last & 3) * ns + s, (last >> 2) & 1, status, kFlagTimeout, site);
     }
 }
 
@@ -95,20 +103,19 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     uint64_t* p_full = tm_empty + C::NBUF;    // [2] P and alpha of a tile written
     uint64_t* d_full = p_full + 2;            // [2] V GEMM of a tile complete
     uint64_t* d_empty = d_full + 2;           // [2] V accumulator read by every compute warp
-    uint64_t* k_full = d_empty + 2;           // [NK]
-    uint64_t* k_empty = k_full + C::NK;
-    uint64_t* v_full = k_empty + C::NK;       // [NV]
-    uint64_t* v_empty = v_full + C::NV;
+    // Round r of a ring slot lands on its barrier of set r % 4: compute warps drift apart by up to
+    // NBUF head groups, more than a ring round, and with four barriers per slot a parity wait can
+    // only alias a round four rounds back, which every reader has long released.
+    uint64_t* k_full = d_empty + 2;           // [4][NK]
+    uint64_t* k_empty = k_full + 4 * C::NK;
+    uint64_t* v_full = k_empty + C::NK;       // [4][NV]
+    uint64_t* v_empty = v_full + 4 * C::NV;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_empty + C::NV);
-    // loads issued per slot (a compute warp first waits for its round to be issued, so that
-    // its parity wait cannot match an earlier round of the slot)
-    volatile uint32_t* k_issued = tmem_holder + 1;
-    volatile uint32_t* v_issued = k_issued + C::NK;
-    float* alpha_s = reinterpret_cast<float*>(tmem_holder + 64);  // [2][4 quarters][HC]
+    float* alpha_s = reinterpret_cast<float*>(tmem_holder + 4);  // [2][4 quarters][HC]
+    auto kf = [&](uint32_t slot, uint32_t round) { return k_full + (round & 3) * C::NK + slot; };
+    auto vf = [&](uint32_t slot, uint32_t round) { return v_full + (round & 3) * C::NV + slot; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x < C::NK) k_issued[threadIdx.x] = 0;
-    if (threadIdx.x < C::NV) v_issued[threadIdx.x] = 0;
     // P starts all zero: each compute warp only ever writes its own block of it
     for (int i = threadIdx.x; i < 2 * C::P_BYTES / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(p_s)[i] = make_uint4(0, 0, 0, 0);
@@ -127,14 +134,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             mbar_init(tm_full + i, 1);
             mbar_init(tm_empty + i, 4);  // the group's warp of each quarter
         }
-        for (int i = 0; i < C::NK; ++i) {
-            mbar_init(k_full + i, 1);
-            mbar_init(k_empty + i, C::HC / C::HPW);  // the group warps of the quarter
-        }
-        for (int i = 0; i < C::NV; ++i) {
-            mbar_init(v_full + i, 1);
-            mbar_init(v_empty + i, 1);  // V GEMM commit
-        }
+        for (int i = 0; i < 4 * C::NK; ++i) mbar_init(k_full + i, 1);
+        for (int i = 0; i < C::NK; ++i) mbar_init(k_empty + i, C::HC / C::HPW);  // the group warps of the quarter
+        for (int i = 0; i < 4 * C::NV; ++i) mbar_init(v_full + i, 1);
+        for (int i = 0; i < C::NV; ++i) mbar_init(v_empty + i, 1);  // V GEMM commit
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -186,18 +189,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     const uint32_t slot = kk_n % C::NK, round = kk_n / C::NK;
                     if (round > 0 && !(ok = mbar_wait(k_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 23)))
                         break;
-                    mbar_expect_tx(k_full + slot, C::K_SLOT);
+                    mbar_expect_tx(kf(slot, round), C::K_SLOT);
                     int tok, outer;
                     tile_coords(p, wk.b, wk.t, tok, outer);
                     tma_load_4d(k_s + size_t(slot) * C::K_SLOT, &lat_map, 0, 0, tok + q * C::QTOK, outer,
-                                k_full + slot, pol_stream);
-                    __threadfence_block();  // the armed barrier phase precedes the published round
-                    k_issued[slot] = round + 1;
+                                kf(slot, round), pol_stream);
                     ++kk_n;
                 }
             }
             // no copy may still be in flight when the CTA exits
-            wait_last_phases(k_full, C::NK, kk_n, p.status, 24);
+            wait_last_phases4(k_full, C::NK, kk_n, p.status, 24);
             wait_last_phases(phi_full, 2, phi_n, p.status, 25);
             if (mq_n > 0) mbar_wait(mq_full, (mq_n - 1) & 1, p.status, kFlagTimeout, 26);
         }
@@ -214,17 +215,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     const uint32_t slot = vk_n % C::NV, round = vk_n / C::NV;
                     if (round > 0 && !(ok = mbar_wait(v_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 27)))
                         break;
-                    mbar_expect_tx(v_full + slot, C::V_SLOT);
+                    mbar_expect_tx(vf(slot, round), C::V_SLOT);
 #pragma unroll
                     for (int pn = 0; pn < C::V_PANELS; ++pn)
                         tma_load_4d(v_s + size_t(slot) * C::V_SLOT + pn * C::PANEL, &lat_map, C::RK + 64 * pn, 0,
-                                    vtok + q * C::QTOK, vouter, v_full + slot, pol_stream);
-                    __threadfence_block();
-                    v_issued[slot] = round + 1;
+                                    vtok + q * C::QTOK, vouter, vf(slot, round), pol_stream);
                     ++vk_n;
                 }
             }
-            wait_last_phases(v_full, C::NV, vk_n, p.status, 28);
+            wait_last_phases4(v_full, C::NV, vk_n, p.status, 28);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -242,7 +241,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 const uint32_t d_tmem = tmem_base + C::VCOL + pb * C::VN;
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t vs = n * 4 + q, slot = vs % C::NV;
-                    if (!mbar_wait(v_full + slot, (vs / C::NV) & 1, p.status, kFlagTimeout, 31)) return false;
+                    if (!mbar_wait(vf(slot, vs / C::NV), (vs / C::NV >> 2) & 1, p.status, kFlagTimeout, 31)) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
@@ -408,8 +407,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             {
                 bool w = true;
                 if (lane == 0) {
-                    w = ok && wait_issued(k_issued + kslot, ks / C::NK + 1, p.status, kFlagTimeout, 41);
-                    w = w && mbar_wait(k_full + kslot, (ks / C::NK) & 1, p.status, kFlagTimeout, 42);
+                    w = ok && mbar_wait(kf(kslot, ks / C::NK), (ks / C::NK >> 2) & 1, p.status, kFlagTimeout, 42);
                 }
                 ok = __shfl_sync(0xffffffffu, w, 0) && ok;
                 __syncwarp();
@@ -497,8 +495,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 const uint32_t vs = tile_n * 4 + qd, vslot = vs % C::NV;
                 bool w = true;
                 if (lane == 0) {
-                    w = ok && wait_issued(v_issued + vslot, vs / C::NV + 1, p.status, kFlagTimeout, 44);
-                    w = w && mbar_wait(v_full + vslot, (vs / C::NV) & 1, p.status, kFlagTimeout, 45);
+                    w = ok && mbar_wait(vf(vslot, vs / C::NV), (vs / C::NV >> 2) & 1, p.status, kFlagTimeout, 45);
                 }
                 ok = __shfl_sync(0xffffffffu, w, 0) && ok;
                 __syncwarp();

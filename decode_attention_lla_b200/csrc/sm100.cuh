@@ -67,21 +67,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
-// Wait (bounded) until a shared-memory counter written by another warp reaches `target`.  A
-// waiter here is ahead of the producer, so after a few polls it sleeps between them and leaves
-// the issue slots to the warps that are working (about 1% faster decode kernels on B200).
-__device__ __forceinline__ bool wait_issued(volatile uint32_t* counter, uint32_t target, uint32_t* status,
-                                            uint32_t timeout_bit, uint32_t site = 0) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (*counter >= target) return true;
-        if (i >= 4) __nanosleep(128);
-        if ((i & 1023u) == 1023u && (*reinterpret_cast<volatile uint32_t*>(status) & timeout_bit)) return false;
-    }
-    atomicCAS(status + 1, 0u, site + 1);
-    atomicOr(status, timeout_bit);
-    return false;
-}
-
 // ---- L2 cache policies --------------------------------------------------------
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
