@@ -700,14 +700,55 @@ def run_full(a, cfg):
     tag = f"bench/{a.workload}/full"
     K = torch.empty(elems, dtype=torch.bfloat16, device=dev)
     V = torch.empty(elems, dtype=torch.bfloat16, device=dev)
-    syn.fill_gaussian_bf16_(K, tag + "/K")
-    syn.fill_gaussian_bf16_(V, tag + "/V")
+    seq_stride = D * TS * cap * H * d
+    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    # The fast path's cache: rebuilt once from a seeded latent store of the workload's codec
+    # (lla_reconstruct_cache), one (layer, loop) slice per call, timed as its own roofline.
+    # Where store and cache do not fit together the cache is filled with seeded Gaussians.
+    recon = None
+    desc = lla.Desc(D, T, H, d, cfg["r_k"], cfg["r_v"], cfg["variant"], cfg["rope_base"], cap + 1)
+    store_b = lla.store_bytes(desc, B, cap)
+    if store_b < torch.cuda.mem_get_info(dev)[0] - (4 << 30):
+        codec_np = syn.seeded_codec(cfg, tag + "/codec")
+        rnd = {k: (syn.round_bf16(v) if k.startswith("w_down") else syn.round_f32(v)) for k, v in codec_np.items()}
+        codec = lla.Codec(desc, rnd["w_down_k"], rnd["w_down_v"], rnd["w_up_k"], rnd["w_up_v"], rnd["mu_k"], rnd["mu_v"])
+        store = torch.empty(store_b // 2, dtype=torch.bfloat16, device=dev)
+        syn.fill_gaussian_bf16_(store, tag + "/latents")
+        loops = [T - 1] if a.final_loop else list(range(T))
+
+        def rebuild():
+            for si, t in enumerate(loops):
+                for layer in range(D):
+                    off = 2 * (layer * TS + si) * cap * H * d
+                    lla.reconstruct_cache(codec, store, B, cap, layer, t, lens, K.data_ptr() + off, V.data_ptr() + off,
+                                          seq_stride, cap)
+
+        rebuild()  # warm-up
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record()
+        rebuild()
+        r1.record()
+        torch.cuda.synchronize()
+        rms = r0.elapsed_time(r1)
+        slices = len(loops) * D
+        per_slice = B * N * H * ((cfg["r_k"] + cfg["r_v"]) * 2 + 2 * d * 2)  # latents read + K, V rows written
+        peak_r, kind_r = measured_peak()
+        ach = per_slice * slices / (rms / 1e3) / 1e9
+        recon = {"kernel": "lla_reconstruct_cache (one (layer, loop) slice per call)", "ms_total": rms,
+                 "ms_per_slice": rms / slices, "slices": slices, "algorithmic_bytes_per_slice": per_slice,
+                 "bound": "hbm", "achieved": ach, "peak": peak_r, "unit": "GB/s", "frac": ach / peak_r,
+                 "peak_source": f"{kind_r} hbm_gbs"}
+        del store
+        codec.close()
+        torch.cuda.empty_cache()
+    else:
+        syn.fill_gaussian_bf16_(K, tag + "/K")
+        syn.fill_gaussian_bf16_(V, tag + "/V")
     q_all = torch.empty(T, D, B, H, d, dtype=torch.float32, device=dev)
     q_all.normal_(generator=syn.torch_generator(tag + "/q", dev))
-    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
     out = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     ws = torch.empty(lla.full_decode_workspace_bytes(H, d, B), dtype=torch.uint8, device=dev)
-    seq_stride = D * TS * cap * H * d
     scale = 1.0 / math.sqrt(d)
 
     def step():
@@ -737,7 +778,10 @@ def run_full(a, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(config_json(cfg, a.workload, 1),
                            step=f"{T}x{D} decode calls over a full bf16 K/V cache (comparator, no LLA)",
-                           cache_gb=2 * elems * 2 / 1e9, loop_slots=TS),
+                           cache_gb=2 * elems * 2 / 1e9, loop_slots=TS,
+                           cache_source="rebuilt from a seeded latent store by lla_reconstruct_cache" if recon
+                           else "seeded Gaussians (store and cache do not fit together)"),
+            "reconstruct": recon,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic_record("full", a.workload),
                          "kernel": "full-cache decode (prologue + decode + combine, per step)",

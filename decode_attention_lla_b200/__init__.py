@@ -79,6 +79,8 @@ _full_decode = _sig("lla_full_decode_attn", _i, [_i, _i, _f, _vp, _vp, ctypes.c_
                                                  _vp, _vp, _sz, _i, _vp])
 _fit_ws = _sig("lla_fit_codec_workspace_bytes", _sz, [_i, _i, _i, _i])
 _fit = _sig("lla_fit_codec", _i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp])
+_reconstruct = _sig("lla_reconstruct_cache", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, ctypes.c_longlong, _i, _i,
+                                                  _vp])
 _decode_self = _sig("lla_decode_attn_self", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _sz,
                                                  ctypes.POINTER(DecodeOpts), _vp])
 
@@ -87,7 +89,7 @@ EXPORTED = ["lla_status_string", "lla_version", "lla_create_codec", "lla_destroy
             "lla_decode_attn_2d", "lla_decode_attn_ex", "lla_workspace_flags", "lla_decode_attn_noalloc",
             "lla_decode_attn_self", "lla_paged_store_bytes", "lla_encode_paged", "lla_decode_attn_paged",
             "lla_full_decode_workspace_bytes", "lla_full_decode_attn", "lla_fit_codec_workspace_bytes",
-            "lla_fit_codec"]
+            "lla_fit_codec", "lla_reconstruct_cache"]
 PAGE_TOKENS = 128
 FLAG_PAGE_INVALID = 4
 FLAG_FIT_BREAKDOWN = 8
@@ -294,6 +296,14 @@ def full_decode_attn(H, d_head, rope_base, k_cache, v_cache, seq_stride, batch, 
     _check(_full_decode(H, d_head, float(rope_base), _ptr(k_cache), _ptr(v_cache), int(seq_stride), batch, max_tokens,
                         _ptr(q), _ptr(q_pos), _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
                         int(workspace_bytes), num_ctas, _stream(stream)), "lla_full_decode_attn")
+
+
+def reconstruct_cache(codec, store, batch, max_tokens, layer, loop, seq_lens, k_cache, v_cache, seq_stride,
+                      cache_tokens, impl=IMPL_AUTO, stream=None):
+    """lla_reconstruct_cache: one (layer, loop) slice of the full K/V cache (keys rotated) rebuilt from
+    the latent store, in the layout full_decode_attn reads."""
+    _check(_reconstruct(codec.handle, _ptr(store), batch, max_tokens, layer, loop, _ptr(seq_lens), _ptr(k_cache),
+                        _ptr(v_cache), int(seq_stride), cache_tokens, impl, _stream(stream)), "lla_reconstruct_cache")
 
 
 def fit_codec_workspace_bytes(problems: int, n: int, S: int, r: int) -> int:

@@ -54,7 +54,8 @@ lla_status dev_alloc(T** p, size_t count) {
 void codec_free(lla_codec* c) {
     if (!c) return;
     void* ptrs[] = {c->w_up_k, c->w_up_v, c->mu_k, c->mu_v, c->bias_k, c->bias_v,
-                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles, c->status, c->w_up_k_t};
+                    c->w_down_k_t, c->w_down_v_t, c->rope_cos, c->rope_sin, c->phi_tiles, c->status, c->w_up_k_t,
+                    c->w_up_k_bf16, c->w_up_v_bf16};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     delete c;
@@ -124,7 +125,8 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
         (st = dev_alloc(&c->bias_k, groups * rk)) || (st = dev_alloc(&c->bias_v, groups * rv)) ||
         (st = dev_alloc(&c->w_down_k_t, groups * rk * S)) || (st = dev_alloc(&c->w_down_v_t, groups * rv * S)) ||
         (st = dev_alloc(&c->rope_cos, nrope)) || (st = dev_alloc(&c->rope_sin, nrope)) ||
-        (st = dev_alloc(&c->status, 4)) || (st = dev_alloc(&c->w_up_k_t, size_t(D) * T * H * (rk + 1) * d))) {
+        (st = dev_alloc(&c->status, 4)) || (st = dev_alloc(&c->w_up_k_t, size_t(D) * T * H * (rk + 1) * d)) ||
+        (st = dev_alloc(&c->w_up_k_bf16, nup_k)) || (st = dev_alloc(&c->w_up_v_bf16, nup_v))) {
         codec_free(c);
         return st;
     }
@@ -173,7 +175,12 @@ lla_status lla_create_codec(lla_codec** out, const lla_codec_desc* desc, const f
                     for (int i = 0; i < d; ++i) o[size_t(n) * d + i] = W[size_t(i) * rk + n];
                 for (int i = 0; i < d; ++i) o[size_t(rk) * d + i] = m[i];
             }
+    std::vector<uint16_t> wup16_k(nup_k), wup16_v(nup_v);
+    for (size_t i = 0; i < nup_k; ++i) wup16_k[i] = f32_to_bf16_rne(w_up_k[i]);
+    for (size_t i = 0; i < nup_v; ++i) wup16_v[i] = f32_to_bf16_rne(w_up_v[i]);
     bool ok = cudaMemcpyAsync(c->w_up_k_t, wupt.data(), wupt.size() * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_up_k_bf16, wup16_k.data(), nup_k * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
+              cudaMemcpyAsync(c->w_up_v_bf16, wup16_v.data(), nup_v * 2, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->w_up_k, w_up_k, nup_k * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->w_up_v, w_up_v, nup_v * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
               cudaMemcpyAsync(c->mu_k, mu_k, nmu * 4, cudaMemcpyHostToDevice, stream) == cudaSuccess &&
@@ -409,6 +416,35 @@ lla_status lla_fit_codec(int problems, int n, int S, int r, const float* X, floa
     if (workspace_bytes < lla_fit_workspace_bytes_impl(problems, n, S, r)) return LLA_ERR_WORKSPACE;
     return lla_fit(problems, n, S, r, X, mu, w_down, sigma, iters == 0 ? 24 : iters, workspace,
                    static_cast<cudaStream_t>(stream));
+}
+
+lla_status lla_reconstruct_cache(const lla_codec* c, const uint16_t* store, int batch, int max_tokens, int layer,
+                                 int loop, const int32_t* seq_lens, uint16_t* k_cache, uint16_t* v_cache,
+                                 long long seq_stride, int cache_tokens, int impl, void* stream) {
+    if (!c || batch < 0 || max_tokens < 0 || layer < 0 || layer >= c->desc.D || loop < 0 || loop >= c->desc.T)
+        return LLA_ERR_INVALID_ARG;
+    if (impl < 0 || impl > 2 || max_tokens > c->desc.max_pos || cache_tokens < max_tokens) return LLA_ERR_INVALID_ARG;
+    if (batch == 0 || max_tokens == 0) return LLA_OK;
+    if (!store || !seq_lens || !k_cache || !v_cache) return LLA_ERR_INVALID_ARG;
+    const long long seq_elems = (long long)c->desc.H * cache_tokens * c->desc.d_head;
+    if (seq_stride < seq_elems || seq_stride % 8 != 0) return LLA_ERR_INVALID_ARG;
+    if (!aligned16(store) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned4(seq_lens))
+        return LLA_ERR_ALIGNMENT;
+    if (impl == 2 && !lla_reconstruct_tc_supported(c)) return LLA_ERR_UNSUPPORTED_SHAPE;
+    lla_reconstruct_call rc;
+    rc.codec = c;
+    rc.store = store;
+    rc.batch = batch;
+    rc.max_tokens = max_tokens;
+    rc.layer = layer;
+    rc.loop = loop;
+    rc.seq_lens = seq_lens;
+    rc.k_cache = k_cache;
+    rc.v_cache = v_cache;
+    rc.seq_stride = seq_stride;
+    rc.cache_tokens = cache_tokens;
+    rc.stream = static_cast<cudaStream_t>(stream);
+    return lla_reconstruct_launch(rc, impl);
 }
 
 lla_status lla_workspace_flags(const void* workspace, uint32_t* flags, void* stream) {

@@ -32,6 +32,10 @@ struct lla_codec {
     // image the tensor-core decode kernel feeds to tcgen05.mma.
     uint16_t* phi_tiles = nullptr;
     int phi_num_tiles = 0;
+    // bf16 copies of W_up (same layouts as w_up_k / w_up_v): the B operands of the tensor-core
+    // reconstruction of a full K/V cache (lla_reconstruct_cache)
+    uint16_t* w_up_k_bf16 = nullptr;
+    uint16_t* w_up_v_bf16 = nullptr;
     // Device status words of the tensor-core encode (bit 2: a bounded wait gave up; word 1:
     // the first wait site that did).
     uint32_t* status = nullptr;
@@ -96,6 +100,21 @@ struct lla_decode_call {
     const float* v_self = nullptr;   // key (pre-RoPE) and value, [batch][H][d_head]
     lla_store_map smap;              // paged store (max_tokens = max_pages * kPageTokens)
 };
+
+// One (layer, loop) slice of a full K/V cache rebuilt from the latent store.
+struct lla_reconstruct_call {
+    const lla_codec* codec;
+    const uint16_t* store;
+    int batch, max_tokens, layer, loop;
+    const int32_t* seq_lens;
+    uint16_t* k_cache;
+    uint16_t* v_cache;
+    long long seq_stride;
+    int cache_tokens;
+    cudaStream_t stream;
+};
+bool lla_reconstruct_tc_supported(const lla_codec* c);
+lla_status lla_reconstruct_launch(const lla_reconstruct_call& rc, int impl);
 
 // ---- bf16 helpers ---------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

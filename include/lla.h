@@ -275,6 +275,31 @@ lla_status lla_full_decode_attn(int H, int d_head, float rope_base, const uint16
                                 void* stream);
 
 /*
+ * lla_reconstruct_cache — the fast path's cache: rebuild the loop-t keys and values of every
+ *   cached token once from the latent store and keep them [LLA summary, "Serving Capacity"],
+ *   for one (layer, loop):
+ *     k_hat_j = RoPE_j(c^K_j W^K_up,t^T + mu^K_t),   v_hat_j = c^V_j W^V_up,t^T + mu^V_t
+ *   [LLA §3 eq. (3); RoPE after reconstruction, "RoPE and reconstruction"], rounded to bf16
+ *   (nearest-even), written in the layout lla_full_decode_attn reads (keys already rotated).
+ *   Either codec variant (2D: head h reconstructs from the token's one latent).
+ *   store      device bf16 latent store (layout of lla_store_bytes), 16-byte aligned
+ *   seq_lens   device int32 [batch]: tokens j < min(seq_lens[b], max_tokens) are written; the
+ *              other rows of the cache are left as they are
+ *   k_cache, v_cache  device bf16, 16-byte aligned: sequence b's head h, token j at element
+ *              b * seq_stride + (h * cache_tokens + j) * d_head; seq_stride a multiple of 8,
+ *              >= H * cache_tokens * d_head; cache_tokens >= max_tokens
+ *   impl       0 = best available, 1 = CUDA-core kernel (any shape), 2 = tcgen05 kernel
+ *              (d_head 128 with r_k/r_v 16/32 or 96/160 per head, or 64/128 for LLA-2D; it
+ *              multiplies by a bf16 copy of W_up, the CUDA-core kernel by the fp32 one)
+ *   Requires max_tokens <= the codec's max_pos (positions of the RoPE table); otherwise
+ *   LLA_ERR_INVALID_ARG.  Asynchronous on `stream`.
+ */
+lla_status lla_reconstruct_cache(const lla_codec* codec, const uint16_t* store, int batch, int max_tokens,
+                                 int layer, int loop, const int32_t* seq_lens, uint16_t* k_cache,
+                                 uint16_t* v_cache, long long seq_stride, int cache_tokens, int impl,
+                                 void* stream);
+
+/*
  * lla_decode_attn_self — decode attention with the current token as a self slot
  *   [LLA §3 eq. (2)-(3)]: a token's latent is written only after its last loop
  *   (eq. (2) encodes the whole loop stack), so while it is being decoded its
