@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--self-slot", action="store_true",
                     help="decode calls attend to the current token's exact K/V as well (lla_decode_attn_self)")
     ap.add_argument("--calib", type=int, default=1024, help="fit mode: calibration stacks per (layer, head, axis)")
+    ap.add_argument("--q-std", type=float, default=1.0,
+                    help="decode mode: queries drawn N(0, q_std^2); 8 spreads the logits by ~2.4 (peaked attention)")
     ap.add_argument("--final-loop", action="store_true",
                     help="full mode: cache only the final loop's K/V and use it for every loop (zero-parameter "
                          "matched-budget baseline: 1/T of the full cache)")
@@ -327,7 +329,7 @@ def run_ours(a, cfg):
     store = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
     syn.fill_gaussian_bf16_(store, tag + "/store")
     q_all = torch.empty(T, D, B, H, d, dtype=torch.float32, device=dev)
-    q_all.normal_(generator=syn.torch_generator(tag + "/q", dev))
+    q_all.normal_(0.0, a.q_std, generator=syn.torch_generator(tag + "/q", dev))
     S = T * d if cfg["variant"] == 0 else T * H * d
     x_shape = (B, D, H, 2, S) if cfg["variant"] == 0 else (B, D, 2, S)
     kv_self = None
@@ -498,7 +500,8 @@ def run_ours(a, cfg):
                                **({"self_slot": "current token's exact K/V attended in every call"}
                                   if kv_self is not None else {}),
                                **({"store": f"paged: {pages} pages of {lla.PAGE_TOKENS} tokens per sequence, "
-                                            "shuffled over the pool"} if table is not None else {})),
+                                            "shuffled over the pool"} if table is not None else {}),
+                               **({"query_std": a.q_std} if a.q_std != 1.0 else {})),
                 "hbm_gbs_per_gpu_step": bytes_per_call(cfg) * T * D / (ms_max / a.steps / 1e3) / 1e9,
                 "roofline": dict(roofline(cfg, kernel_name, kern_ms, a.workload),
                                  timed_launches=f"{len(kern_ms)} of {a.steps * T * D}: every {every}th decode call "
