@@ -42,7 +42,7 @@ DEFAULT_WORKLOAD = "ouro_rho21_b768_n4096"
 LAUNCHES_PER_DECODE = {"simt": 2, "tc": 3}
 LAUNCHES_PER_ENCODE = 1
 KERNEL_SOURCES = {"simt": ["decode_simt.cu", "sm100.cuh"], "tc": ["decode_tc.cu", "decode_tc2d.cuh", "sm100.cuh", "walk.cuh"],
-                  "full": ["decode_full.cu", "sm100.cuh", "walk.cuh"]}
+                  "full": ["decode_full.cu", "sm100.cuh", "walk.cuh"], "recon": ["reconstruct.cu", "sm100.cuh"]}
 
 
 def parse():
@@ -741,7 +741,7 @@ def run_full(a, cfg):
         recon = {"kernel": "lla_reconstruct_cache (one (layer, loop) slice per call)", "ms_total": rms,
                  "ms_per_slice": rms / slices, "slices": slices, "algorithmic_bytes_per_slice": per_slice,
                  "bound": "hbm", "achieved": ach, "peak": peak_r, "unit": "GB/s", "frac": ach / peak_r,
-                 "peak_source": f"{kind_r} hbm_gbs"}
+                 "traffic": traffic_record("recon", a.workload), "peak_source": f"{kind_r} hbm_gbs"}
         del store
         codec.close()
         torch.cuda.empty_cache()
