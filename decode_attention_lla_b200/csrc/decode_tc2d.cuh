@@ -470,9 +470,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 mx[hh] = s2[hh];
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int hh = 0; hh < HPW; ++hh) mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], o));
+            for (int hh = 0; hh < HPW; ++hh) mx[hh] = warp_max_f32(mx[hh]);
             const uint32_t pb = tile_n & 1;
             // P and alpha go to buffer tile_n & 1, last used by tile n - 2, whose V GEMM and
             // readers must be done with it

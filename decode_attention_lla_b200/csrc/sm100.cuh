@@ -67,6 +67,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+// Maximum of v over the 32 lanes of a warp in one instruction (sm_100a: redux.sync on f32);
+// every lane gets the result.  Inputs are finite or -inf here.
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
 // ---- L2 cache policies --------------------------------------------------------
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
