@@ -407,11 +407,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc_decode_kernel(const __grid_c
         long long prev_id = 0;
         bool ok = true;
 
+        // every lane waits on the stage's barrier (no divergent lane-0 branch on the path) and the
+        // warp agrees by one vote
         auto wait_stage = [&](uint32_t slot, uint32_t round) {
-            bool w_ok = true;
-            if (lane == 0) w_ok = ok && mbar_wait(st_full_bar(slot, round), (round >> 2) & 1, p.status, kFlagTimeout, 13);
-            ok = __shfl_sync(0xffffffffu, w_ok, 0) && ok;
-            __syncwarp();  // lane 0's barrier acquire covers the whole warp's reads
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(st_full_bar(slot, round), (round >> 2) & 1, p.status,
+                                                           kFlagTimeout, 13)) && ok;
         };
 
         auto flush = [&](long long id) {
