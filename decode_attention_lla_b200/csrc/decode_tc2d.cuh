@@ -60,6 +60,10 @@ struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
     static_assert(HC * 4 == VN, "V GEMM columns = heads of the item x quarters");
     static_assert(VCOL + 2 * VN <= TMEM_COLS, "TMEM columns");
     static_assert(NV >= 4, "c^V ring");
+    // the c^V producer frees a slot on its tile's d_full phase: the last slot of tile m is refilled
+    // at stage 4m + 3 + NV, which must precede tile m + 2's last stage (4m + 11), or d_full[m & 1]
+    // could be one phase further on than the parity the producer waits for
+    static_assert(NV <= 8, "c^V ring at most two tiles");
     static_assert(SMEM <= kSmemLimit, "shared memory");
     static_assert((6 + 2 * NBUF + 6 + 5 * NK + 5 * NV) * 8 + 16 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
 };
@@ -109,8 +113,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     uint64_t* k_full = d_empty + 2;           // [4][NK]
     uint64_t* k_empty = k_full + 4 * C::NK;
     uint64_t* v_full = k_empty + C::NK;       // [4][NV]
-    uint64_t* v_empty = v_full + 4 * C::NV;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_empty + C::NV);
+    // a c^V slot is free again once its tile's V GEMM is complete: the producer waits on d_full
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_full + 4 * C::NV);
     float* alpha_s = reinterpret_cast<float*>(tmem_holder + 4);  // [2][4 quarters][HC]
     auto kf = [&](uint32_t slot, uint32_t round) { return k_full + (round & 3) * C::NK + slot; };
     auto vf = [&](uint32_t slot, uint32_t round) { return v_full + (round & 3) * C::NV + slot; };
@@ -137,7 +141,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         for (int i = 0; i < 4 * C::NK; ++i) mbar_init(k_full + i, 1);
         for (int i = 0; i < C::NK; ++i) mbar_init(k_empty + i, C::HC / C::HPW);  // the group warps of the quarter
         for (int i = 0; i < 4 * C::NV; ++i) mbar_init(v_full + i, 1);
-        for (int i = 0; i < C::NV; ++i) mbar_init(v_empty + i, 1);  // V GEMM commit
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -213,7 +216,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 tile_coords(p, wk.b, wk.t, vtok, vouter);
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t slot = vk_n % C::NV, round = vk_n / C::NV;
-                    if (round > 0 && !(ok = mbar_wait(v_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 27)))
+                    // the slot's previous tile m: its V GEMM complete (d_full[m & 1], phase m / 2).  The
+                    // producer never runs two phases ahead: it waited for every earlier tile in order.
+                    const uint32_t m = (vk_n - C::NV) / 4;
+                    if (round > 0 && !(ok = mbar_wait(d_full + (m & 1), (m >> 1) & 1, p.status, kFlagTimeout, 27)))
                         break;
                     mbar_expect_tx(vf(slot, round), C::V_SLOT);
 #pragma unroll
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            uint32_t phi_n = 0, mq_n = 0, mq_commits = 0, tile_n = 0, v_commits = 0, v_next = 0;
+            uint32_t phi_n = 0, mq_n = 0, mq_commits = 0, tile_n = 0, v_next = 0;
             int prev_key = -1;
             bool ok = true;
             const uint32_t phi_addr = smem_u32(phi_s), mq_addr = smem_u32(mq_s);
@@ -238,11 +244,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 const uint32_t pb = n & 1, use = n >> 1;
                 if (!mbar_wait(p_full + pb, use & 1, p.status, kFlagTimeout, 29)) return false;
                 if (use > 0 && !mbar_wait(d_empty + pb, (use - 1) & 1, p.status, kFlagTimeout, 30)) return false;
+                tc_fence_after();  // the accumulator's readers (tcgen05.ld) are done with it
                 const uint32_t d_tmem = tmem_base + C::VCOL + pb * C::VN;
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t vs = n * 4 + q, slot = vs % C::NV;
+                    // TMA-filled operands: the barrier wait alone orders them before the MMA
                     if (!mbar_wait(vf(slot, vs / C::NV), (vs / C::NV >> 2) & 1, p.status, kFlagTimeout, 31)) return false;
-                    tc_fence_after();
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int kk = 2 * q + k2;  // sixteen-token step of the tile
@@ -252,10 +259,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                                                               uint32_t(kk >> 2) * (C::VN * 128) + uint32_t(kk & 3) * 32);
                         mma_f16_ss(d_tmem, ad, bd, C::IDESC_V, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(v_empty + slot);
-                    ++v_commits;
                 }
-                mma_commit(d_full + pb);
+                mma_commit(d_full + pb);  // also frees the tile's four c^V slots
                 return true;
             };
             // V GEMMs of every tile before `end` not issued yet
@@ -281,7 +286,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 const uint32_t pb = phi_n & 1;
                 if (!(ok = mbar_wait(phi_full + pb, (phi_n >> 1) & 1, p.status, kFlagTimeout, 33))) break;
                 ++phi_n;
-                tc_fence_after();
                 const uint32_t phi_buf = phi_addr + pb * C::PHI_BYTES;
                 for (int g = 0; g < C::GPC && ok; ++g) {
                     const uint32_t gi = tile_n * C::GPC + g;
@@ -310,7 +314,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             }
             // the commits' arrivals land in shared memory: see them complete before the CTA exits
             wait_last_phases(phi_empty, 2, phi_n, p.status, 35);
-            wait_last_phases(v_empty, C::NV, v_commits, p.status, 36);
             if (mq_commits > 0) mbar_wait(mq_empty, (mq_commits - 1) & 1, p.status, kFlagTimeout, 37);
         }
     } else {
