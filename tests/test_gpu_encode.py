@@ -44,6 +44,8 @@ CASES = [
     dict(D=3, T=4, H=4, d_head=128, r_k=16, r_v=32, variant=0, n=200, B=2, N=160, layers=(1, 2)),
     dict(D=1, T=4, H=2, d_head=128, r_k=96, r_v=160, variant=0, n=130, B=1, N=130, layers=(0, 1)),
     dict(D=1, T=32, H=2, d_head=128, r_k=96, r_v=160, variant=0, n=70, B=2, N=64, layers=(0, 1)),
+    # several 256-token items of the wide codec, the last one ragged
+    dict(D=3, T=4, H=2, d_head=128, r_k=96, r_v=160, variant=0, n=700, B=2, N=400, layers=(1, 3)),
     dict(D=2, T=2, H=4, d_head=16, r_k=12, r_v=20, variant=1, n=150, B=2, N=100, layers=(0, 2)),
     dict(D=1, T=4, H=16, d_head=128, r_k=64, r_v=128, variant=1, n=100, B=1, N=128, layers=(0, 1)),
     # T = 1: per-loop MLA, the head-axis latent of one loop
