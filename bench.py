@@ -657,12 +657,13 @@ def run_encode(a, cfg):
         lla.encode(codec, x, n, 0, D, seq, tok, store, slots, n)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(a.steps):
-        seq.fill_(i % slots)
-        lla.encode(codec, x, n, 0, D, seq, tok, store, slots, n)
-    e1.record()
-    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        e0.record()
+        for i in range(a.steps):
+            seq.fill_(i % slots)
+            lla.encode(codec, x, n, 0, D, seq, tok, store, slots, n)
+        e1.record()
+        torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.steps
     in_bytes = int(np.prod(x_shape)) * 2
     peak, kind = measured_peak()
@@ -672,7 +673,9 @@ def run_encode(a, cfg):
             "config": dict(config_json(cfg, a.workload, 1), step=f"encode {n} tokens x {D} layers"),
             "roofline": {"bound": "hbm", "achieved": in_bytes / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                          "frac": in_bytes / (ms / 1e3) / 1e9 / peak, "traffic": None, "kernel": "lla encode",
-                         "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": in_bytes}}
+                         "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_launch": in_bytes,
+                         "latent_bytes_written": n * D * (H if cfg["variant"] == 0 else 1) * (rk + rv) * 2},
+            "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
     codec.close()
     return 0
