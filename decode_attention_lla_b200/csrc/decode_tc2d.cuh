@@ -237,8 +237,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             uint32_t phi_n = 0, mq_n = 0, mq_commits = 0, tile_n = 0, v_next = 0;
             int prev_key = -1;
             bool ok = true;
-            const uint32_t phi_addr = smem_u32(phi_s), mq_addr = smem_u32(mq_s);
-            const uint32_t p_addr = smem_u32(p_s), v_addr = smem_u32(v_s);
+            // operand descriptors: built once; an operand's start address moves by adding its byte
+            // offset / 16 to the descriptor (the 14-bit address field cannot carry: shared memory
+            // addresses stay below 2^18)
+            const uint64_t phi_desc = sw128_kmajor_desc(smem_u32(phi_s)), mq_desc = sw128_kmajor_desc(smem_u32(mq_s));
+            const uint64_t p_desc = sw128_kmajor_desc(smem_u32(p_s));
+            const uint64_t v_desc = sw128_mnmajor_desc(smem_u32(v_s), C::PANEL, 1024);
             // V GEMM of tile n: D[pb] = sum over its 8 sixteen-token steps of (C^V)^T . P
             auto issue_v = [&](uint32_t n) -> bool {
                 const uint32_t pb = n & 1, use = n >> 1;
@@ -253,10 +257,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int kk = 2 * q + k2;  // sixteen-token step of the tile
-                        const uint64_t ad = sw128_mnmajor_desc(v_addr + slot * C::V_SLOT + k2 * (16 * 128),
-                                                               C::PANEL, 1024);
-                        const uint64_t bd = sw128_kmajor_desc(p_addr + pb * C::P_BYTES +
-                                                              uint32_t(kk >> 2) * (C::VN * 128) + uint32_t(kk & 3) * 32);
+                        const uint64_t ad = v_desc + ((slot * C::V_SLOT + k2 * (16 * 128)) >> 4);
+                        const uint64_t bd = p_desc + ((pb * C::P_BYTES + uint32_t(kk >> 2) * (C::VN * 128) +
+                                                       uint32_t(kk & 3) * 32) >> 4);
                         mma_f16_ss(d_tmem, ad, bd, C::IDESC_V, kk > 0 ? 1u : 0u);
                     }
                 }
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 const uint32_t pb = phi_n & 1;
                 if (!(ok = mbar_wait(phi_full + pb, (phi_n >> 1) & 1, p.status, kFlagTimeout, 33))) break;
                 ++phi_n;
-                const uint32_t phi_buf = phi_addr + pb * C::PHI_BYTES;
+                const uint64_t phi_d = phi_desc + ((pb * C::PHI_BYTES) >> 4);
                 for (int g = 0; g < C::GPC && ok; ++g) {
                     const uint32_t gi = tile_n * C::GPC + g;
                     const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
@@ -294,11 +297,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + buf * C::BUF_COLS;
 #pragma unroll
+                    const uint64_t mq_d = mq_desc + ((g * C::MQ_GROUP_BYTES) >> 4);
                     for (int kk = 0; kk < C::DH / 16; ++kk) {
                         const uint32_t koff = uint32_t(kk & 3) * 32;
-                        const uint64_t ad = sw128_kmajor_desc(phi_buf + uint32_t(kk >> 2) * (kTile * 128) + koff);
-                        const uint64_t bd = sw128_kmajor_desc(mq_addr + g * C::MQ_GROUP_BYTES +
-                                                              uint32_t(kk >> 2) * (C::NG * 128) + koff);
+                        const uint64_t ad = phi_d + ((uint32_t(kk >> 2) * (kTile * 128) + koff) >> 4);
+                        const uint64_t bd = mq_d + ((uint32_t(kk >> 2) * (C::NG * 128) + koff) >> 4);
                         mma_f16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(tm_full + buf);
