@@ -65,7 +65,7 @@ struct Cfg2 : HeadGroups<DH_, RK_, RV_, H_> {
     // could be one phase further on than the parity the producer waits for
     static_assert(NV <= 8, "c^V ring at most two tiles");
     static_assert(SMEM <= kSmemLimit, "shared memory");
-    static_assert((6 + 2 * NBUF + 6 + 5 * NK + 5 * NV) * 8 + 16 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
+    static_assert((6 + 2 * NBUF + 6 + 5 * NK + 4) * 8 + 16 + 2 * 4 * HC * 4 <= BAR_BYTES, "barrier area");
 };
 
 // Wait for the last phase of each of `ns` ring barriers after `count` uses in ring order.
@@ -112,12 +112,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
     // only alias a round four rounds back, which every reader has long released.
     uint64_t* k_full = d_empty + 2;           // [4][NK]
     uint64_t* k_empty = k_full + 4 * C::NK;
-    uint64_t* v_full = k_empty + C::NK;       // [4][NV]
-    // a c^V slot is free again once its tile's V GEMM is complete: the producer waits on d_full
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(v_full + 4 * C::NV);
+    // c^V of tile n (its four quarter slots) lands on vt_full[n % 4]; a slot is free again once its
+    // tile's V GEMM is complete: the producer waits on d_full
+    uint64_t* vt_full = k_empty + C::NK;      // [4]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(vt_full + 4);
     float* alpha_s = reinterpret_cast<float*>(tmem_holder + 4);  // [2][4 quarters][HC]
     auto kf = [&](uint32_t slot, uint32_t round) { return k_full + (round & 3) * C::NK + slot; };
-    auto vf = [&](uint32_t slot, uint32_t round) { return v_full + (round & 3) * C::NV + slot; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // P starts all zero: each compute warp only ever writes its own block of it
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         }
         for (int i = 0; i < 4 * C::NK; ++i) mbar_init(k_full + i, 1);
         for (int i = 0; i < C::NK; ++i) mbar_init(k_empty + i, C::HC / C::HPW);  // the group warps of the quarter
-        for (int i = 0; i < 4 * C::NV; ++i) mbar_init(v_full + i, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(vt_full + i, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -209,11 +209,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
         // ------------------------------------------------------------ c^V loads
         if (elect_one()) {
             const uint64_t pol_stream = policy_evict_normal();
-            uint32_t vk_n = 0;
+            uint32_t vk_n = 0, vt_n = 0;
             bool ok = true;
-            for (; wk.valid() && ok; wk.next()) {
+            for (; wk.valid() && ok; wk.next(), ++vt_n) {
                 int vtok, vouter;
                 tile_coords(p, wk.b, wk.t, vtok, vouter);
+                // the tile's four quarters on one barrier.  Its previous phase (tile vt_n - 4) is
+                // complete: refilling the slots of tile vt_n - 1 needed tile vt_n - 2's V GEMM done
+                uint64_t* vbar = vt_full + (vt_n & 3);
+                mbar_expect_tx(vbar, 4 * C::V_SLOT);
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t slot = vk_n % C::NV, round = vk_n / C::NV;
                     // the slot's previous tile m: its V GEMM complete (d_full[m & 1], phase m / 2).  The
@@ -221,20 +225,24 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     const uint32_t m = (vk_n - C::NV) / 4;
                     if (round > 0 && !(ok = mbar_wait(d_full + (m & 1), (m >> 1) & 1, p.status, kFlagTimeout, 27)))
                         break;
-                    mbar_expect_tx(vf(slot, round), C::V_SLOT);
 #pragma unroll
                     for (int pn = 0; pn < C::V_PANELS; ++pn)
                         tma_load_4d(v_s + size_t(slot) * C::V_SLOT + pn * C::PANEL, &lat_map, C::RK + 64 * pn, 0,
-                                    vtok + q * C::QTOK, vouter, vf(slot, round), pol_stream);
+                                    vtok + q * C::QTOK, vouter, vbar, pol_stream);
                     ++vk_n;
                 }
             }
-            wait_last_phases4(v_full, C::NV, vk_n, p.status, 28);
+            // no copy in flight at exit: the last (up to) four tiles' barriers complete.  A tile
+            // cut short by a failed wait has bytes that never arrive: its wait gives up (bounded).
+            for (uint32_t t = vt_n > 4 ? vt_n - 4 : 0; t < vt_n; ++t)
+                mbar_wait(vt_full + (t & 3), (t >> 2) & 1, p.status, kFlagTimeout, 28);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
             uint32_t phi_n = 0, mq_n = 0, mq_commits = 0, tile_n = 0, v_next = 0;
+            uint32_t v_slot = 0;            // c^V slot of quarter 0 of tile v_next: (4 v_next) % NV
+            uint32_t sbuf = 0, suse = 0;    // score buffer of the next head group and its use count
             int prev_key = -1;
             bool ok = true;
             // operand descriptors: built once; an operand's start address moves by adding its byte
@@ -250,10 +258,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 if (use > 0 && !mbar_wait(d_empty + pb, (use - 1) & 1, p.status, kFlagTimeout, 30)) return false;
                 tc_fence_after();  // the accumulator's readers (tcgen05.ld) are done with it
                 const uint32_t d_tmem = tmem_base + C::VCOL + pb * C::VN;
+                // TMA-filled operands: the barrier wait alone orders them before the MMA
+                if (!mbar_wait(vt_full + (n & 3), (n >> 2) & 1, p.status, kFlagTimeout, 31)) return false;
+#pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t vs = n * 4 + q, slot = vs % C::NV;
-                    // TMA-filled operands: the barrier wait alone orders them before the MMA
-                    if (!mbar_wait(vf(slot, vs / C::NV), (vs / C::NV >> 2) & 1, p.status, kFlagTimeout, 31)) return false;
+                    const uint32_t slot = v_slot + q < C::NV ? v_slot + q : v_slot + q - C::NV;
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int kk = 2 * q + k2;  // sixteen-token step of the tile
@@ -264,6 +273,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                     }
                 }
                 mma_commit(d_full + pb);  // also frees the tile's four c^V slots
+                v_slot = v_slot + 4 < C::NV ? v_slot + 4 : v_slot + 4 - C::NV;
                 return true;
             };
             // V GEMMs of every tile before `end` not issued yet
@@ -291,13 +301,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                 ++phi_n;
                 const uint64_t phi_d = phi_desc + ((pb * C::PHI_BYTES) >> 4);
                 for (int g = 0; g < C::GPC && ok; ++g) {
-                    const uint32_t gi = tile_n * C::GPC + g;
-                    const uint32_t buf = gi % C::NBUF, use = gi / C::NBUF;
+                    const uint32_t buf = sbuf, use = suse;
+                    if (++sbuf == C::NBUF) {
+                        sbuf = 0;
+                        ++suse;
+                    }
                     if (use > 0 && !(ok = mbar_wait(tm_empty + buf, (use - 1) & 1, p.status, kFlagTimeout, 34))) break;
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + buf * C::BUF_COLS;
-#pragma unroll
                     const uint64_t mq_d = mq_desc + ((g * C::MQ_GROUP_BYTES) >> 4);
+#pragma unroll
                     for (int kk = 0; kk < C::DH / 16; ++kk) {
                         const uint32_t koff = uint32_t(kk & 3) * 32;
                         const uint64_t ad = phi_d + ((uint32_t(kk >> 2) * (kTile * 128) + koff) >> 4);
@@ -496,10 +509,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             if (g == 0 && nv < 32) {
                 // rows past the context may hold any bits, and 0 * NaN is not 0: clear them in
                 // the c^V slot before the V GEMM reads it
-                const uint32_t vs = tile_n * 4 + qd, vslot = vs % C::NV;
+                const uint32_t vslot = (tile_n * 4 + qd) % C::NV;
                 bool w = true;
                 if (lane == 0) {
-                    w = ok && mbar_wait(vf(vslot, vs / C::NV), (vs / C::NV >> 2) & 1, p.status, kFlagTimeout, 45);
+                    w = ok && mbar_wait(vt_full + (tile_n & 3), (tile_n >> 2) & 1, p.status, kFlagTimeout, 45);
                 }
                 ok = __shfl_sync(0xffffffffu, w, 0) && ok;
                 __syncwarp();
