@@ -188,13 +188,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
                              phi_full + pb, pol_keep);
                     ++phi_n;
                 }
+                int tok, outer;
+                tile_coords(p, wk.b, wk.t, tok, outer);
                 for (int q = 0; q < 4; ++q) {
                     const uint32_t slot = kk_n % C::NK, round = kk_n / C::NK;
                     if (round > 0 && !(ok = mbar_wait(k_empty + slot, (round - 1) & 1, p.status, kFlagTimeout, 23)))
                         break;
                     mbar_expect_tx(kf(slot, round), C::K_SLOT);
-                    int tok, outer;
-                    tile_coords(p, wk.b, wk.t, tok, outer);
                     tma_load_4d(k_s + size_t(slot) * C::K_SLOT, &lat_map, 0, 0, tok + q * C::QTOK, outer,
                                 kf(slot, round), pol_stream);
                     ++kk_n;
@@ -254,8 +254,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) tc2d_decode_kernel(const __grid
             // V GEMM of tile n: D[pb] = sum over its 8 sixteen-token steps of (C^V)^T . P
             auto issue_v = [&](uint32_t n) -> bool {
                 const uint32_t pb = n & 1, use = n >> 1;
+                // p_full also says that the accumulator D[pb] is free: every compute warp waits for
+                // d_empty[pb] (its readers of tile n - 2 done) before it writes P of tile n
                 if (!mbar_wait(p_full + pb, use & 1, p.status, kFlagTimeout, 29)) return false;
-                if (use > 0 && !mbar_wait(d_empty + pb, (use - 1) & 1, p.status, kFlagTimeout, 30)) return false;
                 tc_fence_after();  // the accumulator's readers (tcgen05.ld) are done with it
                 const uint32_t d_tmem = tmem_base + C::VCOL + pb * C::VN;
                 // TMA-filled operands: the barrier wait alone orders them before the MMA
