@@ -381,7 +381,9 @@ __global__ void __launch_bounds__(kThreads) encode_tc_wide_kernel(const __grid_c
             prefetch_tensormap(&xmap);
             prefetch_tensormap(&wkmap);
             prefetch_tensormap(&wvmap);
-            const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
+            // stacks at normal L2 priority: the 256-byte promotion of a 128-byte row brings the
+            // token's next chunk, which the stage after next reads (evict-first measured 2.5% slower)
+            const uint64_t pol_x = policy_evict_normal(), pol_w = policy_evict_last();
             int issued = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < p.nitems && ok; it += gridDim.x) {
