@@ -18,7 +18,11 @@
 // the codec's decode table) and the head's mu_t, so that four epilogue warps (thread = token
 // row) add mu, rotate key pairs (i, i + d/2), round to bf16 and write the rows without a global
 // load on their path.  (Reading each row's cos/sin and mu from global memory inside the epilogue
-// loop measured 1.03 ms per slice at ratio 4, batch 32 x 4096: 0.32 of the copy peak.)
+// loop measured 1.03 ms per slice at ratio 4, batch 32 x 4096: 0.32 of the copy peak.)  A warp
+// gathers 64 outputs of each of its 32 rows in shared memory and writes them as whole 128-byte
+// lines, four rows per store instruction: a 16-byte piece of 32 rows per instruction kept the
+// write requests, not DRAM, the limit (0.577 ms per slice against 0.248 ms with the stores
+// left out).
 //   warp 0  TMA producer   warp 1  TMEM allocator + MMA issuer   warps 2-5  epilogue
 // W_up enters the GEMM as bf16 (a copy the codec keeps) and the rotation uses fp16 cos/sin: the
 // cache itself is bf16, and both roundings are of the same order as the cache's own or below.
@@ -66,7 +70,11 @@ struct RCfg {
     static constexpr int PHI_BYTES = kTok * kDh * 2;
     static constexpr int AUX_BYTES = PHI_BYTES + 2 * kDh * 4;
     static constexpr int NST = 4;
-    static constexpr int SMEM = 1024 + NST * STAGE + 2 * AUX_BYTES + 1024;
+    // per epilogue warp: 32 rows x 128 bytes, where a half-row of output is gathered so that the
+    // warp writes whole 128-byte lines (four rows per store instruction) instead of one 16-byte
+    // piece of each of 32 rows
+    static constexpr int XPOSE_BYTES = 4 * 32 * 128;
+    static constexpr int SMEM = 1024 + NST * STAGE + 2 * AUX_BYTES + XPOSE_BYTES + 1024;
     static constexpr int ACC_COLS = 2 * kDh;         // K then V accumulator
     static constexpr int TMEM_COLS = 2 * ACC_COLS;   // two buffers
     static constexpr uint32_t IDESC = idesc_bf16_f32(128, kDh, false, false);
@@ -145,7 +153,8 @@ __global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* aux_s = smem + C::NST * C::STAGE;  // [2 items][Phi image | mu^K_t | mu^V_t]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(aux_s + 2 * C::AUX_BYTES);
+    uint8_t* xpose_s = aux_s + 2 * C::AUX_BYTES;  // [4 epilogue warps][32 rows][128 B]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xpose_s + C::XPOSE_BYTES);
     uint64_t* full = bars;                     // [NST]
     uint64_t* empty = bars + C::NST;           // [NST]
     uint64_t* acc_full = bars + 2 * C::NST;    // [2]
@@ -264,6 +273,12 @@ __global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_c
     } else {
         // epilogue: warps 2..5 -> TMEM lane quarters 2, 3, 0, 1; thread = token row of the tile
         const int qd = warp & 3, row = 32 * qd + lane;
+        // this warp's gather rows: row r's 16-byte chunk c at r * 128 + (c ^ (r % 8)) * 16, so that
+        // eight consecutive rows' chunk c fall in eight different bank groups
+        uint8_t* xp = xpose_s + (warp - 2) * (32 * 128);
+        auto gather = [&](int c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+            *reinterpret_cast<uint4*>(xp + lane * 128 + ((c ^ (lane & 7)) << 4)) = make_uint4(w0, w1, w2, w3);
+        };
         bool ok = true;
         int j = 0;
         for (int it = blockIdx.x; it < p.nitems && ok; it += gridDim.x) {
@@ -271,9 +286,23 @@ __global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_c
             if (!item_of(p, it, b, tile, h, len)) continue;
             const int buf = j & 1, use = j >> 1;
             ++j;
-            const int tok = tile * kTok + row;
-            const bool write = tok < len;
-            const size_t orow = size_t(b) * p.seq_stride + (size_t(h) * p.cache_tokens + (write ? tok : 0)) * kDh;
+            // rows of this warp: tile rows 32 qd .. 32 qd + 31, row r of the tile at
+            // rbase + r * d_head (keys and values alike), written only below the sequence length
+            const size_t rbase = size_t(b) * p.seq_stride + (size_t(h) * p.cache_tokens + size_t(tile) * kTok) * kDh;
+            const int nrows = len - tile * kTok;  // rows of the tile below the length (> 0)
+            // the gathered half-row (64 outputs, 128 bytes) of each row, out as whole lines:
+            // lane l stores chunk l % 8 of row 4 s + l / 8
+            auto flush = [&](uint16_t* cache, int half) {
+                __syncwarp();
+#pragma unroll
+                for (int s4 = 0; s4 < 8; ++s4) {
+                    const int r = 4 * s4 + (lane >> 3), c = lane & 7;
+                    const uint4 v = *reinterpret_cast<const uint4*>(xp + r * 128 + ((c ^ (r & 7)) << 4));
+                    if (32 * qd + r < nrows)
+                        *reinterpret_cast<uint4*>(cache + rbase + size_t(32 * qd + r) * kDh + half * 64 + c * 8) = v;
+                }
+                __syncwarp();
+            };
             bool w = mbar_wait(aux_full + buf, use & 1, p.status, kFlagTimeout, 87);
             w = w && mbar_wait(acc_full + buf, use & 1, p.status, kFlagTimeout, 84);
             ok = __all_sync(0xffffffffu, w);
@@ -284,47 +313,48 @@ __global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_c
             const float* muv = muk + kDh;
             const uint32_t taddr = tmem + buf * C::ACC_COLS + (uint32_t(32 * qd) << 16);
             // keys: pairs (i, i + 64) rotated by the token's position; cos and sin of the row's
-            // position from the Phi image (k < 64: cos, k >= 64: sin; 128-byte swizzle)
+            // position from the Phi image (k < 64: cos, k >= 64: sin; 128-byte swizzle).  One half
+            // of the rotated row per pass (x cos - y sin, then y cos + x sin), each gathered and out
 #pragma unroll 1
-            for (int c0 = 0; c0 < kDh / 2; c0 += 16) {
-                float x[16], y[16];
-                tmem_ld<16>(taddr + c0, x);
-                tmem_ld<16>(taddr + c0 + kDh / 2, y);
-                float cv[16], sv[16];
-                phi16(cv, phi, row, c0);
-                phi16(sv, phi, row, c0 + kDh / 2);
-                tmem_wait_ld();
-                if (write) {
-                    uint32_t lo[8], hi[8];
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int c0 = 0; c0 < kDh / 2; c0 += 16) {
+                    float x[16], y[16];
+                    tmem_ld<16>(taddr + c0, x);
+                    tmem_ld<16>(taddr + c0 + kDh / 2, y);
+                    float cv[16], sv[16];
+                    phi16(cv, phi, row, c0);
+                    phi16(sv, phi, row, c0 + kDh / 2);
+                    tmem_wait_ld();
+                    uint32_t o[8];
 #pragma unroll
                     for (int e = 0; e < 16; e += 2) {
                         const float x0 = x[e] + muk[c0 + e], y0 = y[e] + muk[c0 + e + kDh / 2];
                         const float x1 = x[e + 1] + muk[c0 + e + 1], y1 = y[e + 1] + muk[c0 + e + 1 + kDh / 2];
-                        lo[e / 2] = pack_bf16x2(x0 * cv[e] - y0 * sv[e], x1 * cv[e + 1] - y1 * sv[e + 1]);
-                        hi[e / 2] = pack_bf16x2(y0 * cv[e] + x0 * sv[e], y1 * cv[e + 1] + x1 * sv[e + 1]);
+                        o[e / 2] = half == 0 ? pack_bf16x2(x0 * cv[e] - y0 * sv[e], x1 * cv[e + 1] - y1 * sv[e + 1])
+                                             : pack_bf16x2(y0 * cv[e] + x0 * sv[e], y1 * cv[e + 1] + x1 * sv[e + 1]);
                     }
-                    uint4* kl = reinterpret_cast<uint4*>(p.k_cache + orow + c0);
-                    uint4* kh = reinterpret_cast<uint4*>(p.k_cache + orow + c0 + kDh / 2);
-                    kl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                    kl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-                    kh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    kh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+                    gather(c0 / 8, o[0], o[1], o[2], o[3]);
+                    gather(c0 / 8 + 1, o[4], o[5], o[6], o[7]);
                 }
+                flush(p.k_cache, half);
             }
-            // values
+            // values, one half-row at a time
 #pragma unroll 1
-            for (int c0 = 0; c0 < kDh; c0 += 16) {
-                float v[16];
-                tmem_ld<16>(taddr + kDh + c0, v);
-                tmem_wait_ld();
-                if (write) {
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int c0 = 0; c0 < kDh / 2; c0 += 16) {
+                    const int col = half * (kDh / 2) + c0;
+                    float v[16];
+                    tmem_ld<16>(taddr + kDh + col, v);
+                    tmem_wait_ld();
                     uint32_t o[8];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) o[e / 2] = pack_bf16x2(v[e] + muv[c0 + e], v[e + 1] + muv[c0 + e + 1]);
-                    uint4* vo = reinterpret_cast<uint4*>(p.v_cache + orow + c0);
-                    vo[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                    vo[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                    for (int e = 0; e < 16; e += 2) o[e / 2] = pack_bf16x2(v[e] + muv[col + e], v[e + 1] + muv[col + e + 1]);
+                    gather(c0 / 8, o[0], o[1], o[2], o[3]);
+                    gather(c0 / 8 + 1, o[4], o[5], o[6], o[7]);
                 }
+                flush(p.v_cache, half);
             }
             tc_fence_before();
             __syncwarp();
