@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -274,11 +275,22 @@ def roofline(cfg, kernel_name, kern_ms, workload):
     return r
 
 
+_COMMENT = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+
+
+def _code_only(src):
+    """The source with its comments removed (string literals kept) and blank runs collapsed:
+    a traffic record stays valid across comment-only edits."""
+    out = _COMMENT.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", src)
+    return "\n".join(ln.rstrip() for ln in out.splitlines() if ln.strip())
+
+
 def kernel_sha(kernel):
+    """SHA-256 of the kernel's sources without comments (the code the traffic was taken on)."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "decode_attention_lla_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "decode_attention_lla_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

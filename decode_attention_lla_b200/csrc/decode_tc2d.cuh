@@ -19,10 +19,11 @@
 //               quarter slots (one 128-byte swizzled row per token).
 //   warp 1      TMEM allocator and MMA issuer: per tile the score GEMMs of every head
 //               group, then the V GEMM of the previous tile (its P is complete by then).
-//   warp 2      TMA: c^V quarter slots (two 64-wide swizzled panels per token).
-//   warps 3-18  compute: one warp per (TMEM lane quarter, head of the item).  Per tile:
-//               score, softmax, P and alpha into shared memory, then the previous tile's
-//               V GEMM result into its accumulators.
+//   warp 2      TMA: c^V quarter slots (two 64-wide swizzled panels per token), the four
+//               quarters of a tile on one barrier.
+//   warps 3-10  compute: one warp per (TMEM lane quarter, head group of the item; two heads
+//               per group).  Per tile: score, softmax, P and alpha into shared memory, then
+//               the previous tile's V GEMM result into its accumulators.
 // Every wait is bounded and sets a status bit on timeout.
 
 template <int DH_, int RK_, int RV_, int H_>

@@ -73,3 +73,13 @@ def test_defaults(monkeypatch):
     a = bench.parse()
     assert a.gpus == 1 and a.steps >= 1 and a.warmup >= 3 and a.kernel_sample >= 1
     assert a.workload == "ouro_rho21_b768_n4096"
+
+
+def test_kernel_sha_ignores_comments_only():
+    """A traffic record stays valid across comment-only edits of its kernel's sources, and not
+    across code edits (string literals count as code)."""
+    base = 'int a = 1; // note\n/* block\n comment */ f("// kept");\n'
+    assert bench._code_only(base) == bench._code_only(base.replace("// note", "// another note"))
+    assert bench._code_only(base) == bench._code_only(base.replace("block", "longer block"))
+    assert bench._code_only(base) != bench._code_only(base.replace("a = 1", "a = 2"))
+    assert bench._code_only(base) != bench._code_only(base.replace('"// kept"', '"// changed"'))
