@@ -401,13 +401,16 @@ def run_ours(a, cfg):
         """One step through host buffers: every call's query (and self-slot K/V) goes up from pinned
         memory and its output comes back, and the step's new-token stacks go up.  The copies run on
         a copy-in and a copy-out stream beside the compute stream, into double-buffered device
-        slots ordered by events, so the transfers of neighbouring calls overlap the decode."""
+        slots ordered by events, so the transfers of neighbouring calls overlap the decode.  The
+        stacks (all layers of every sequence's new token, the largest copy of the step) go up in
+        one piece per call behind that call's query, so no query waits behind all of them."""
         cs = torch.cuda.current_stream(dev)
         cin, cout = host["cin"], host["cout"]
-        with torch.cuda.stream(cin):  # this step's new-token stacks, once the last encode read them
+        xs_host, xs_dev = host["x"].view(-1), x_new.view(-1)
+        ncalls = T * D
+        piece = -(-xs_host.numel() // ncalls)
+        with torch.cuda.stream(cin):  # the stacks' slots are free once the last encode read them
             cin.wait_event(host["x_free"])
-            x_new.copy_(host["x"], non_blocking=True)
-            host["x_ready"].record(cin)
         k = 0
         for t in range(T):
             for layer in range(D):
@@ -418,6 +421,12 @@ def run_ours(a, cfg):
                     if kv_self is not None:
                         host["kv_dev"][sl].copy_(host["kv"][t, layer], non_blocking=True)
                     host["ready"][sl].record(cin)
+                    a0 = k * piece
+                    if a0 < xs_host.numel():
+                        b0 = min(a0 + piece, xs_host.numel())
+                        xs_dev[a0:b0].copy_(xs_host[a0:b0], non_blocking=True)
+                    if k == ncalls - 1:
+                        host["x_ready"].record(cin)
                 cs.wait_event(host["ready"][sl])
                 cs.wait_event(host["out_free"][sl])  # its output two calls back has been copied out
                 ks = vs = None
