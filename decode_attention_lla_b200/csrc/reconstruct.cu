@@ -149,7 +149,7 @@ __device__ __forceinline__ bool item_of(const RParams& p, int it, int& b, int& t
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_constant__ RMaps maps, RParams p) {
+__global__ void __launch_bounds__(kThreads, 1) reconstruct_tc_kernel(const __grid_constant__ RMaps maps, RParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* aux_s = smem + C::NST * C::STAGE;  // [2 items][Phi image | mu^K_t | mu^V_t]
@@ -313,32 +313,34 @@ __global__ void __launch_bounds__(kThreads) reconstruct_tc_kernel(const __grid_c
             const float* muv = muk + kDh;
             const uint32_t taddr = tmem + buf * C::ACC_COLS + (uint32_t(32 * qd) << 16);
             // keys: pairs (i, i + 64) rotated by the token's position; cos and sin of the row's
-            // position from the Phi image (k < 64: cos, k >= 64: sin; 128-byte swizzle).  One half
-            // of the rotated row per pass (x cos - y sin, then y cos + x sin), each gathered and out
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            // position from the Phi image (k < 64: cos, k >= 64: sin; 128-byte swizzle).  The
+            // first halves are gathered as they come, the second ones kept in registers until
+            // those are out (one CTA per SM: the launch bounds leave room for them)
+            uint32_t hi[kDh / 4];
 #pragma unroll
-                for (int c0 = 0; c0 < kDh / 2; c0 += 16) {
-                    float x[16], y[16];
-                    tmem_ld<16>(taddr + c0, x);
-                    tmem_ld<16>(taddr + c0 + kDh / 2, y);
-                    float cv[16], sv[16];
-                    phi16(cv, phi, row, c0);
-                    phi16(sv, phi, row, c0 + kDh / 2);
-                    tmem_wait_ld();
-                    uint32_t o[8];
+            for (int c0 = 0; c0 < kDh / 2; c0 += 16) {
+                float x[16], y[16];
+                tmem_ld<16>(taddr + c0, x);
+                tmem_ld<16>(taddr + c0 + kDh / 2, y);
+                float cv[16], sv[16];
+                phi16(cv, phi, row, c0);
+                phi16(sv, phi, row, c0 + kDh / 2);
+                tmem_wait_ld();
+                uint32_t lo[8];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        const float x0 = x[e] + muk[c0 + e], y0 = y[e] + muk[c0 + e + kDh / 2];
-                        const float x1 = x[e + 1] + muk[c0 + e + 1], y1 = y[e + 1] + muk[c0 + e + 1 + kDh / 2];
-                        o[e / 2] = half == 0 ? pack_bf16x2(x0 * cv[e] - y0 * sv[e], x1 * cv[e + 1] - y1 * sv[e + 1])
-                                             : pack_bf16x2(y0 * cv[e] + x0 * sv[e], y1 * cv[e + 1] + x1 * sv[e + 1]);
-                    }
-                    gather(c0 / 8, o[0], o[1], o[2], o[3]);
-                    gather(c0 / 8 + 1, o[4], o[5], o[6], o[7]);
+                for (int e = 0; e < 16; e += 2) {
+                    const float x0 = x[e] + muk[c0 + e], y0 = y[e] + muk[c0 + e + kDh / 2];
+                    const float x1 = x[e + 1] + muk[c0 + e + 1], y1 = y[e + 1] + muk[c0 + e + 1 + kDh / 2];
+                    lo[e / 2] = pack_bf16x2(x0 * cv[e] - y0 * sv[e], x1 * cv[e + 1] - y1 * sv[e + 1]);
+                    hi[c0 / 2 + e / 2] = pack_bf16x2(y0 * cv[e] + x0 * sv[e], y1 * cv[e + 1] + x1 * sv[e + 1]);
                 }
-                flush(p.k_cache, half);
+                gather(c0 / 8, lo[0], lo[1], lo[2], lo[3]);
+                gather(c0 / 8 + 1, lo[4], lo[5], lo[6], lo[7]);
             }
+            flush(p.k_cache, 0);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) gather(c, hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+            flush(p.k_cache, 1);
             // values, one half-row at a time
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
