@@ -285,6 +285,13 @@ def _code_only(src):
     return "\n".join(ln.rstrip() for ln in out.splitlines() if ln.strip())
 
 
+def upload_pieces(numel: int, ncalls: int) -> list:
+    """[begin, end) element ranges of the step's new-token stacks that go up behind each of the
+    step's ncalls queries: equal pieces (the last ones shorter or empty) that cover [0, numel)."""
+    piece = -(-numel // ncalls) if ncalls > 0 else numel
+    return [(min(k * piece, numel), min((k + 1) * piece, numel)) for k in range(ncalls)]
+
+
 def kernel_sha(kernel):
     """SHA-256 of the kernel's sources without comments (the code the traffic was taken on)."""
     h = hashlib.sha256()
@@ -408,7 +415,7 @@ def run_ours(a, cfg):
         cin, cout = host["cin"], host["cout"]
         xs_host, xs_dev = host["x"].view(-1), x_new.view(-1)
         ncalls = T * D
-        piece = -(-xs_host.numel() // ncalls)
+        pieces = upload_pieces(xs_host.numel(), ncalls)
         with torch.cuda.stream(cin):  # the stacks' slots are free once the last encode read them
             cin.wait_event(host["x_free"])
         k = 0
@@ -421,9 +428,8 @@ def run_ours(a, cfg):
                     if kv_self is not None:
                         host["kv_dev"][sl].copy_(host["kv"][t, layer], non_blocking=True)
                     host["ready"][sl].record(cin)
-                    a0 = k * piece
-                    if a0 < xs_host.numel():
-                        b0 = min(a0 + piece, xs_host.numel())
+                    a0, b0 = pieces[k]
+                    if b0 > a0:
                         xs_dev[a0:b0].copy_(xs_host[a0:b0], non_blocking=True)
                     if k == ncalls - 1:
                         host["x_ready"].record(cin)

@@ -83,3 +83,16 @@ def test_kernel_sha_ignores_comments_only():
     assert bench._code_only(base) == bench._code_only(base.replace("block", "longer block"))
     assert bench._code_only(base) != bench._code_only(base.replace("a = 1", "a = 2"))
     assert bench._code_only(base) != bench._code_only(base.replace('"// kept"', '"// changed"'))
+
+
+@pytest.mark.parametrize("numel,ncalls", [(604 * 2**20, 96), (7, 96), (96, 96), (1000, 7), (0, 4)])
+def test_stack_upload_pieces_cover_the_stacks_once(numel, ncalls):
+    """The e2e step's new-token stacks go up in one piece per call: together the pieces cover
+    every element exactly once, in order."""
+    pieces = bench.upload_pieces(numel, ncalls)
+    assert len(pieces) == ncalls
+    pos = 0
+    for a, b in pieces:
+        assert a == pos and b >= a
+        pos = b
+    assert pos == numel
